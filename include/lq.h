@@ -1,0 +1,198 @@
+/*
+ * liblq: windowed INT8 recurrent-state decode for gated delta-rule linear
+ * attention on NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * The method (LeapQuant, arXiv 2609.38166; "LeapQuant: Efficient Linear
+ * Attention with Accurate Recurrent State Quantization", section "Abstract
+ * (arXiv)"): each (sequence, head) pair of a Gated DeltaNet (GDN) or Kimi
+ * Delta Attention (KDA) layer keeps a d_v x d_k recurrent state S.  The state
+ * is stored as 8-bit codes and is quantized only once per window of W tokens;
+ * within a window, outputs come from the fixed low-bit state together with
+ * high-precision buffered updates.  The largest outlier rows and columns of
+ * the state are kept in FP32 as Compensator Tokens that share the update path
+ * of real tokens, and the remaining residual is smoothed before it is
+ * quantized.
+ *
+ * Recurrences (the published GDN rule; for KDA the per-key-channel gate
+ * multiplies the key side):
+ *   GDN: S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *   KDA: S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *   o_t = S_t q_t.
+ * The gate is passed as g_t = log(alpha_t).  q is used as given (no 1/sqrt(d)
+ * scaling).
+ *
+ * Stored window-start state per (sequence, head): codes Q (int8, d_v x d_k),
+ * row scales sigma (FP32, d_v), column smoothing factors s (FP32, d_k) and
+ * compensators C = sum_c v_c k_c^T (FP32 rank-1 pairs: a row compensator is
+ * (e_i, S[i,:]), a column compensator is (S[:,j], e_j)).  Decoded state:
+ * S~_ij = sigma_i Q_ij s_j + C_ij.
+ *
+ * Conventions for every call:
+ *  - Memory.  The caller owns all device memory.  It allocates one workspace
+ *    of lq_workspace_bytes() bytes (256-byte aligned) and passes device
+ *    pointers; liblq allocates nothing on the device.  A handle owns only host
+ *    metadata.  Inputs are read during the call's kernels and not retained.
+ *  - Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ *    device work is enqueued on it, asynchronously; no call synchronizes except
+ *    lq_device_status().
+ *  - Errors.  Every call returns an lq_status.  Errors found on the host are
+ *    returned at once and leave the state untouched; the text of the last one
+ *    on the calling thread is lq_last_error_string().  Errors found on the
+ *    device (a gate sum out of the safe range, a bounded wait that expired)
+ *    are recorded in the workspace's error word and reported by
+ *    lq_device_status().  No kernel traps or asserts.
+ *  - Window phase.  All sequences of a handle share one window phase: a
+ *    handle counts buffered tokens (lq_window_fill) on the host.
+ *  - Threads.  A handle must not be used by two threads at once.
+ */
+#ifndef LQ_H
+#define LQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LQ_API __attribute__((visibility("default")))
+#else
+#define LQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lq_status {
+    LQ_OK = 0,
+    LQ_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad handle, bad field   */
+    LQ_ERR_UNSUPPORTED = 2,  /* valid request outside the compiled kernels        */
+    LQ_ERR_WORKSPACE = 3,    /* workspace too small or misaligned                 */
+    LQ_ERR_WINDOW_FULL = 4,  /* decode with W tokens buffered: flush first        */
+    LQ_ERR_RANGE = 5,        /* device: gate sum outside the safe range           */
+    LQ_ERR_CUDA = 6,         /* a CUDA runtime call failed (text has the reason)  */
+    LQ_ERR_DEVICE = 7,       /* device: another error recorded in the error word  */
+    LQ_ERR_STATE = 8         /* call out of order (e.g. decode before prefill)    */
+} lq_status;
+
+enum { LQ_GATE_SCALAR = 0 /* GDN */, LQ_GATE_CHANNEL = 1 /* KDA */ };
+enum {
+    LQ_MODE_WINDOW = 0,  /* windowed INT8 state (the method)                 */
+    LQ_MODE_NAIVE = 1,   /* per-token requantized INT8 state (comparator)     */
+    LQ_MODE_FP32 = 2     /* FP32 state, plain recurrence (comparator)         */
+};
+enum { LQ_SELECT_L2 = 0, LQ_SELECT_MAXABS = 1 };
+enum { LQ_DTYPE_F32 = 0, LQ_DTYPE_BF16 = 1 };
+
+/* Device error codes in the workspace error word (lq_layout.err, int32[0]). */
+enum { LQ_DEVERR_NONE = 0, LQ_DEVERR_RANGE = 1, LQ_DEVERR_TIMEOUT = 2 };
+
+typedef struct lq_config {
+    int32_t batch;        /* sequences, >= 1                                     */
+    int32_t heads;        /* heads per sequence, >= 1                            */
+    int32_t d_k;          /* key channels: 64 or 128                             */
+    int32_t d_v;          /* value channels: equal to d_k                        */
+    int32_t window;       /* W, tokens per window, 1..4096 (windowed mode)       */
+    int32_t n_comp_rows;  /* compensator rows, 0..16 (windowed mode)             */
+    int32_t n_comp_cols;  /* compensator columns, 0..16 (windowed mode)          */
+    int32_t gate;         /* LQ_GATE_SCALAR or LQ_GATE_CHANNEL                   */
+    int32_t mode;         /* LQ_MODE_*                                           */
+    int32_t smooth;       /* 1: column smoothing before quantization (windowed)  */
+    int32_t select;       /* compensator ranking: LQ_SELECT_L2 or _MAXABS        */
+    int32_t in_dtype;     /* dtype of q, k, v: LQ_DTYPE_BF16 or LQ_DTYPE_F32     */
+} lq_config;
+
+/*
+ * Byte offsets of the regions of a workspace (each 256-byte aligned), for
+ * callers that inspect or checkpoint the state.  N = batch * heads, units in
+ * (sequence, head) order; absent regions have offset LQ_ABSENT.
+ */
+#define LQ_ABSENT ((size_t)-1)
+typedef struct lq_layout {
+    size_t total_bytes;
+    size_t err;           /* int32[64]: [0] LQ_DEVERR_*, [1] unit, [2] detail     */
+    size_t codes;         /* int8  [N][d_v][d_k]                 window, naive    */
+    size_t row_scale;     /* f32   [N][d_v]       sigma          window, naive    */
+    size_t col_smooth;    /* f32   [N][d_k]       s              window           */
+    size_t comp_index;    /* int32 [N][comp_index_stride]: rows then columns      */
+    size_t comp_row_vec;  /* f32   [N][n_comp_rows][d_k]  k of row compensators   */
+    size_t comp_col_vec;  /* f32   [N][n_comp_cols][d_v]  v of column comps       */
+    size_t gate_sum;      /* f64   [N][1 (GDN) or d_k (KDA)]: sum of g this window*/
+    size_t buf_delta;     /* f32   [N][window][d_v]  buffered delta_j             */
+    size_t buf_key;       /* GDN: in_dtype [N][window][d_k] k_j;
+                             KDA: f32 [N][window][d_k] k_j * exp(-G_j)            */
+    size_t buf_gate;      /* f64   [N][window_pad] G_j (GDN only)                 */
+    size_t state_f32;     /* f32   [N][d_v][d_k]                  FP32 mode        */
+    int32_t comp_index_stride;  /* n_comp_rows + n_comp_cols rounded up to 4      */
+    int32_t window_pad;         /* window rounded up to 2                          */
+} lq_layout;
+
+typedef struct lq_state_s *lq_handle;
+
+/* Bytes of device workspace a config needs; 0 if the config is invalid. */
+LQ_API size_t lq_workspace_bytes(const lq_config *cfg);
+
+/* Fill *out with the workspace layout of a valid config. */
+LQ_API lq_status lq_workspace_layout(const lq_config *cfg, lq_layout *out);
+
+/*
+ * Create a handle over a caller-owned workspace (d_workspace: device pointer,
+ * 256-byte aligned, `bytes` >= lq_workspace_bytes(cfg)).  Host-only: touches
+ * no device memory.  The state is undefined until lq_prefill_state().
+ */
+LQ_API lq_status lq_state_create(const lq_config *cfg, void *d_workspace, size_t bytes, lq_handle *out);
+
+/*
+ * Ingest a prefilled FP32 state and start the first window (the state is
+ * quantized once per window, at its end; the end of the prefill is the start
+ * of the first window).
+ * d_S0: device FP32 [batch][heads][d_v][d_k], or NULL for an all-zero state.
+ *   windowed: the codec (compensator extraction, smoothing, per-row INT8);
+ *   naive:    per-row INT8 without compensators or smoothing;
+ *   FP32:     a copy.
+ * Clears the error word, the gate sums and the window buffer.
+ */
+LQ_API lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream);
+
+/*
+ * One decode token for every (sequence, head): the output is formed from the
+ * INT8 window-start state plus the FP32 buffered updates of the window.
+ * Device inputs, unit-major [batch][heads][.], 16-byte aligned:
+ *   d_q, d_k: [.][d_k], d_v: [.][d_v] in cfg.in_dtype;
+ *   d_g: log alpha, f32 [.] (GDN) or [.][d_k] (KDA);  d_beta: f32 [.];
+ * output d_o: f32 [.][d_v], o_t = S_t q_t.
+ * Windowed mode reads the INT8 window-start state once, adds the buffered
+ * corrections, appends (delta_t, key_t, G_t) to the buffer and writes no
+ * state; it returns LQ_ERR_WINDOW_FULL when W tokens are already buffered.
+ * Naive mode updates and requantizes the INT8 state; FP32 mode updates it.
+ */
+LQ_API lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, const void *d_v,
+                         const float *d_g, const float *d_beta, float *d_o, void *stream);
+
+/*
+ * End the window (windowed mode; a no-op returning LQ_OK otherwise): rebuild
+ * the state in FP32 from the window-start state and the buffered updates,
+ * take the new Compensator Tokens (largest rows, then columns), smooth the
+ * residual and requantize it to per-row INT8; empty the buffer.  Allowed with
+ * any number of buffered tokens, including none.
+ */
+LQ_API lq_status lq_window_flush(lq_handle h, void *stream);
+
+/* Tokens buffered in the current window (0..W); -1 for a bad handle. */
+LQ_API int32_t lq_window_fill(lq_handle h);
+
+/*
+ * Synchronize `stream` and read the device error word: LQ_OK, LQ_ERR_RANGE or
+ * LQ_ERR_DEVICE (detail in lq_last_error_string()).
+ */
+LQ_API lq_status lq_device_status(lq_handle h, void *stream);
+
+/* Release the handle (host metadata only; the workspace stays the caller's). */
+LQ_API lq_status lq_state_destroy(lq_handle h);
+
+/* Text of the last error on the calling thread ("" if none). */
+LQ_API const char *lq_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LQ_H */

@@ -119,8 +119,8 @@ static int argmax_free(const float *score, const unsigned char *taken, int n)
 }
 
 /*
- * The state codec, applied once per window at its end ([abs]: "quantizes the
- * state only once at its end") and once to the prefilled state.
+ * The state codec, applied once per window, at its end ([abs]: the state is
+ * quantized a single time per window), and once to the prefilled state.
  *
  * Input:  S, the dense FP64 state (d_v x d_k, row-major, d_k contiguous).
  * Output: the stored window-start state and, in place of S, its decoded value
@@ -128,17 +128,18 @@ static int argmax_free(const float *score, const unsigned char *taken, int n)
  *
  * All decisions are taken in FP32, the precision of the stored state:
  *  0. R = fp32(S).
- *  1. Compensator Tokens ([abs]: "retains the state's largest outliers as a few
- *     high-precision Compensator Tokens"; [news]: "outlier rows and columns",
- *     kept in FP16/FP32; reading: FP32).  First n_rows rows, ranked on R by
+ *  1. Compensator Tokens ([abs]: the largest outliers of the state stay in
+ *     high precision as a few Compensator Tokens; [news]: the outliers are
+ *     whole rows and columns, kept in FP16/FP32; reading: FP32).  First n_rows rows, ranked on R by
  *     L2 norm (reading; max-abs with select=1), each kept as the rank-1 pair
  *     (v = e_i, k = R[i,:]) and zeroed in R.  Then n_cols columns, ranked on
  *     the row-zeroed R, each kept as (v = R[:,j], k = e_j) and zeroed.
  *     Scores are FP32 sums in index order; ties go to the lower index.
- *  2. Smoothing ([abs]: "smooth the remaining residual before quantization"):
+ *  2. Smoothing ([abs]: the residual left after the compensators is smoothed
+ *     before it is quantized):
  *     m_j = max_i |R_ij|, s_j = sqrt(m_j) rounded to FP32; reading: s_j = 1
  *     where m_j = 0.  Without smoothing s_j = 1.
- *  3. Per-row symmetric INT8 ([abs]: "8-bit recurrent-state quantization"):
+ *  3. Per-row symmetric INT8 ([abs]: the state is held in 8 bits):
  *     R'_ij = R_ij / s_j, sigma_i = max_j |R'_ij| / 127,
  *     Q_ij = clamp(rint(R'_ij / sigma_i), -127, 127) with ties to even;
  *     reading: Q_i = 0 where sigma_i = 0.
@@ -253,16 +254,16 @@ int lqo_num_encodings(const lqo_params *p, int T)
 
 /*
  * One head through T tokens.
- *   FP32 mode:     the plain recurrence from S0 ([news]: "the baseline is FP32
- *                  inference").
+ *   FP32 mode:     the plain recurrence from S0 ([news]: FP32 inference is
+ *                  the baseline).
  *   Windowed mode: the state is encoded from S0, then in every window the
  *                  recurrence runs densely from the decoded window-start state
  *                  and is re-encoded after tokens W, 2W, ... ([abs]).  The
  *                  buffered form a fast implementation uses reaches exactly
  *                  these outputs; this oracle never uses it.
  *   Naive mode:    the state is re-encoded after every token, with no
- *                  compensators and no smoothing ([news]: "naive per-token
- *                  quantization").
+ *                  compensators and no smoothing ([news]: the per-token
+ *                  quantization the paper compares against).
  * Arrays: q,k [T][d_k]; v [T][d_v]; g [T][1 or d_k]; beta [T]; o [T][d_v].
  * S_final (may be NULL) receives the state after the last token (decoded,
  * after any flush at T).  The *_snap arrays (each may be NULL) receive every

@@ -1,0 +1,294 @@
+// liblq C ABI: config validation, workspace layout, handles and launches.
+// The declarations and the contract of every entry point are in include/lq.h.
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "lq.h"
+#include "lq_kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+lq_status fail(lq_status code, const std::string &why) {
+    g_last_error = why;
+    return code;
+}
+
+constexpr uint32_t kMagic = 0x4c515354u;  // "LQST"
+constexpr int kMaxComp = 16;
+constexpr int kMaxWindow = 4096;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool validate(const lq_config *c, std::string *why) {
+    if (c == nullptr) { *why = "config is NULL"; return false; }
+    if (c->batch < 1 || c->heads < 1) { *why = "batch and heads must be >= 1"; return false; }
+    if ((long long)c->batch * c->heads > (1LL << 24)) { *why = "batch * heads must be <= 2^24"; return false; }
+    if (c->d_k != c->d_v) { *why = "d_k must equal d_v"; return false; }
+    if (c->d_k != 64 && c->d_k != 128) { *why = "d_k must be 64 or 128"; return false; }
+    if (c->gate != LQ_GATE_SCALAR && c->gate != LQ_GATE_CHANNEL) { *why = "gate must be LQ_GATE_SCALAR or LQ_GATE_CHANNEL"; return false; }
+    if (c->mode != LQ_MODE_WINDOW && c->mode != LQ_MODE_NAIVE && c->mode != LQ_MODE_FP32) { *why = "mode must be one of LQ_MODE_*"; return false; }
+    if (c->in_dtype != LQ_DTYPE_F32 && c->in_dtype != LQ_DTYPE_BF16) { *why = "in_dtype must be LQ_DTYPE_F32 or LQ_DTYPE_BF16"; return false; }
+    if (c->mode == LQ_MODE_WINDOW) {
+        if (c->window < 1 || c->window > kMaxWindow) { *why = "window must be in 1..4096"; return false; }
+        if (c->n_comp_rows < 0 || c->n_comp_rows > kMaxComp || c->n_comp_cols < 0 || c->n_comp_cols > kMaxComp) {
+            *why = "n_comp_rows and n_comp_cols must be in 0..16"; return false;
+        }
+        if (c->smooth != 0 && c->smooth != 1) { *why = "smooth must be 0 or 1"; return false; }
+        if (c->select != LQ_SELECT_L2 && c->select != LQ_SELECT_MAXABS) { *why = "select must be LQ_SELECT_L2 or LQ_SELECT_MAXABS"; return false; }
+    }
+    return true;
+}
+
+void compute_layout(const lq_config *c, lq_layout *L) {
+    const size_t N = (size_t)c->batch * c->heads, d = (size_t)c->d_k;
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> size_t {
+        if (bytes == 0) return LQ_ABSENT;
+        off = align256(off);
+        const size_t r = off;
+        off += bytes;
+        return r;
+    };
+    lq_layout z;
+    z.total_bytes = 0;
+    z.err = z.codes = z.row_scale = z.col_smooth = z.comp_index = z.comp_row_vec = z.comp_col_vec = LQ_ABSENT;
+    z.gate_sum = z.buf_delta = z.buf_key = z.buf_gate = z.state_f32 = LQ_ABSENT;
+    z.comp_index_stride = 0;
+    z.window_pad = 0;
+    *L = z;
+    L->err = take(256);
+    if (c->mode == LQ_MODE_FP32) {
+        L->state_f32 = take(N * d * d * 4);
+    } else if (c->mode == LQ_MODE_NAIVE) {
+        L->codes = take(N * d * d);
+        L->row_scale = take(N * d * 4);
+    } else {
+        const int ncomp = c->n_comp_rows + c->n_comp_cols;
+        L->comp_index_stride = ((ncomp + 3) / 4) * 4;
+        L->window_pad = ((c->window + 1) / 2) * 2;
+        const size_t gd = (c->gate == LQ_GATE_CHANNEL) ? d : 1;
+        const size_t key_b = (c->gate == LQ_GATE_CHANNEL || c->in_dtype == LQ_DTYPE_F32) ? 4 : 2;
+        L->codes = take(N * d * d);
+        L->row_scale = take(N * d * 4);
+        L->col_smooth = take(N * d * 4);
+        L->comp_index = take(N * (size_t)L->comp_index_stride * 4);
+        L->comp_row_vec = take(N * (size_t)c->n_comp_rows * d * 4);
+        L->comp_col_vec = take(N * (size_t)c->n_comp_cols * d * 4);
+        L->gate_sum = take(N * gd * 8);
+        L->buf_delta = take(N * (size_t)c->window * d * 4);
+        L->buf_key = take(N * (size_t)c->window * d * key_b);
+        if (c->gate == LQ_GATE_SCALAR) L->buf_gate = take(N * (size_t)L->window_pad * 8);
+    }
+    L->total_bytes = align256(off);
+}
+
+template <typename T>
+T *region(unsigned char *base, size_t off) {
+    return off == LQ_ABSENT ? nullptr : reinterpret_cast<T *>(base + off);
+}
+
+lq_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(LQ_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+}  // namespace
+
+struct lq_state_s {
+    uint32_t magic;
+    lq_config cfg;
+    lq_layout lay;
+    unsigned char *ws;
+    int32_t n_buf;
+    int prefilled;
+};
+
+namespace {
+
+bool check_handle(lq_handle h) { return h != nullptr && h->magic == kMagic; }
+
+lq::Views views(lq_handle h) {
+    lq::Views v;
+    unsigned char *b = h->ws;
+    const lq_layout &L = h->lay;
+    v.err = region<int32_t>(b, L.err);
+    v.codes = region<int8_t>(b, L.codes);
+    v.row_scale = region<float>(b, L.row_scale);
+    v.col_smooth = region<float>(b, L.col_smooth);
+    v.comp_index = region<int32_t>(b, L.comp_index);
+    v.comp_row_vec = region<float>(b, L.comp_row_vec);
+    v.comp_col_vec = region<float>(b, L.comp_col_vec);
+    v.gate_sum = region<double>(b, L.gate_sum);
+    v.buf_delta = region<float>(b, L.buf_delta);
+    v.buf_key = region<void>(b, L.buf_key);
+    v.buf_gate = region<double>(b, L.buf_gate);
+    v.state_f32 = region<float>(b, L.state_f32);
+    v.comp_index_stride = L.comp_index_stride;
+    v.window = h->cfg.window;
+    v.window_pad = L.window_pad;
+    v.n_comp_rows = h->cfg.mode == LQ_MODE_WINDOW ? h->cfg.n_comp_rows : 0;
+    v.n_comp_cols = h->cfg.mode == LQ_MODE_WINDOW ? h->cfg.n_comp_cols : 0;
+    v.units = h->cfg.batch * h->cfg.heads;
+    return v;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lq_workspace_bytes(const lq_config *cfg) {
+    std::string why;
+    if (!validate(cfg, &why)) {
+        g_last_error = why;
+        return 0;
+    }
+    lq_layout L;
+    compute_layout(cfg, &L);
+    return L.total_bytes;
+}
+
+lq_status lq_workspace_layout(const lq_config *cfg, lq_layout *out) {
+    std::string why;
+    if (out == nullptr) return fail(LQ_ERR_INVALID_ARG, "layout output is NULL");
+    if (!validate(cfg, &why)) return fail(LQ_ERR_INVALID_ARG, why);
+    compute_layout(cfg, out);
+    return LQ_OK;
+}
+
+lq_status lq_state_create(const lq_config *cfg, void *d_workspace, size_t bytes, lq_handle *out) {
+    std::string why;
+    if (out == nullptr) return fail(LQ_ERR_INVALID_ARG, "handle output is NULL");
+    *out = nullptr;
+    if (!validate(cfg, &why)) return fail(LQ_ERR_INVALID_ARG, why);
+    if (d_workspace == nullptr) return fail(LQ_ERR_WORKSPACE, "workspace is NULL");
+    if (!aligned(d_workspace, 256)) return fail(LQ_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    lq_layout L;
+    compute_layout(cfg, &L);
+    if (bytes < L.total_bytes)
+        return fail(LQ_ERR_WORKSPACE, "workspace has " + std::to_string(bytes) + " bytes, needs " +
+                                          std::to_string(L.total_bytes));
+    lq_state_s *h = new (std::nothrow) lq_state_s;
+    if (h == nullptr) return fail(LQ_ERR_INVALID_ARG, "out of host memory");
+    h->magic = kMagic;
+    h->cfg = *cfg;
+    h->lay = L;
+    h->ws = static_cast<unsigned char *>(d_workspace);
+    h->n_buf = 0;
+    h->prefilled = 0;
+    *out = h;
+    return LQ_OK;
+}
+
+lq_status lq_state_destroy(lq_handle h) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    h->magic = 0;
+    delete h;
+    return LQ_OK;
+}
+
+int32_t lq_window_fill(lq_handle h) { return check_handle(h) ? h->n_buf : -1; }
+
+lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    if (d_S0 != nullptr && !aligned(d_S0, 16)) return fail(LQ_ERR_INVALID_ARG, "S0 must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const lq_config &c = h->cfg;
+    const size_t N = (size_t)c.batch * c.heads, d = (size_t)c.d_k;
+    lq::Views v = views(h);
+    cudaError_t e = cudaMemsetAsync(v.err, 0, 256, s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+    if (c.mode == LQ_MODE_FP32) {
+        e = d_S0 ? cudaMemcpyAsync(v.state_f32, d_S0, N * d * d * 4, cudaMemcpyDeviceToDevice, s)
+                 : cudaMemsetAsync(v.state_f32, 0, N * d * d * 4, s);
+        if (e != cudaSuccess) return cuda_fail(e, "loading the FP32 state");
+    } else {
+        lq::EncodeArgs a;
+        a.w = v;
+        a.S0 = d_S0;
+        a.from_buffer = 0;
+        a.n_buf = 0;
+        const bool win = (c.mode == LQ_MODE_WINDOW);
+        a.n_rows = win ? c.n_comp_rows : 0;
+        a.n_cols = win ? c.n_comp_cols : 0;
+        a.smooth = win ? c.smooth : 0;
+        a.select = win ? c.select : LQ_SELECT_L2;
+        e = lq::launch_encode(a, c.d_k, c.gate, c.in_dtype, s);
+        if (e != cudaSuccess) return cuda_fail(e, "launching the encode kernel");
+    }
+    h->n_buf = 0;
+    h->prefilled = 1;
+    return LQ_OK;
+}
+
+lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, const void *d_v, const float *d_g,
+                         const float *d_beta, float *d_o, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    if (!d_q || !d_k || !d_v || !d_g || !d_beta || !d_o) return fail(LQ_ERR_INVALID_ARG, "NULL input or output");
+    if (!aligned(d_q, 16) || !aligned(d_k, 16) || !aligned(d_v, 16))
+        return fail(LQ_ERR_INVALID_ARG, "q, k, v must be 16-byte aligned");
+    const lq_config &c = h->cfg;
+    if (!aligned(d_g, c.gate == LQ_GATE_CHANNEL ? 16 : 4) || !aligned(d_beta, 4) || !aligned(d_o, 4))
+        return fail(LQ_ERR_INVALID_ARG, "g, beta, o misaligned (g per-channel: 16 bytes; others: 4)");
+    if (!h->prefilled) return fail(LQ_ERR_STATE, "decode before lq_prefill_state");
+    if (c.mode == LQ_MODE_WINDOW && h->n_buf >= c.window)
+        return fail(LQ_ERR_WINDOW_FULL, "window holds W tokens: call lq_window_flush first");
+    lq::DecodeArgs a;
+    a.w = views(h);
+    a.q = d_q; a.k = d_k; a.v = d_v; a.g = d_g; a.beta = d_beta; a.o = d_o;
+    a.n_buf = h->n_buf;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (c.mode == LQ_MODE_WINDOW) e = lq::launch_decode_window(a, c.d_k, c.gate, c.in_dtype, s);
+    else if (c.mode == LQ_MODE_NAIVE) e = lq::launch_decode_naive(a, c.d_k, c.gate, c.in_dtype, s);
+    else e = lq::launch_decode_fp32(a, c.d_k, c.gate, c.in_dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the decode kernel");
+    if (c.mode == LQ_MODE_WINDOW) h->n_buf += 1;
+    return LQ_OK;
+}
+
+lq_status lq_window_flush(lq_handle h, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    const lq_config &c = h->cfg;
+    if (c.mode != LQ_MODE_WINDOW) return LQ_OK;
+    if (!h->prefilled) return fail(LQ_ERR_STATE, "flush before lq_prefill_state");
+    lq::EncodeArgs a;
+    a.w = views(h);
+    a.S0 = nullptr;
+    a.from_buffer = 1;
+    a.n_buf = h->n_buf;
+    a.n_rows = c.n_comp_rows;
+    a.n_cols = c.n_comp_cols;
+    a.smooth = c.smooth;
+    a.select = c.select;
+    cudaError_t e = lq::launch_encode(a, c.d_k, c.gate, c.in_dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launching the flush kernel");
+    h->n_buf = 0;
+    return LQ_OK;
+}
+
+lq_status lq_device_status(lq_handle h, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "synchronizing the stream");
+    int32_t word[3] = {0, 0, 0};
+    e = cudaMemcpy(word, h->ws + h->lay.err, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
+    if (word[0] == LQ_DEVERR_NONE) return LQ_OK;
+    char buf[160];
+    if (word[0] == LQ_DEVERR_RANGE) {
+        snprintf(buf, sizeof buf, "gate sum outside +-80 at unit %d, key channel %d: flush more often", word[1], word[2]);
+        return fail(LQ_ERR_RANGE, buf);
+    }
+    snprintf(buf, sizeof buf, "device error %d at unit %d (detail %d)", word[0], word[1], word[2]);
+    return fail(LQ_ERR_DEVICE, buf);
+}
+
+const char *lq_last_error_string(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

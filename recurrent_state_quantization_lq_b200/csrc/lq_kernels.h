@@ -1,0 +1,39 @@
+// Host-side launchers of the liblq kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lq_common.cuh"
+
+namespace lq {
+
+struct EncodeArgs {
+    Views w;
+    const float *S0;   // prefill source [N][d][d], or nullptr for zeros (prefill only)
+    int from_buffer;   // 1: window flush (stored state + buffer); 0: prefill
+    int n_buf;         // buffered tokens (flush)
+    int n_rows;        // compensator rows to extract
+    int n_cols;        // compensator columns to extract
+    int smooth;        // column smoothing on/off
+    int select;        // LQ_SELECT_*
+};
+
+struct DecodeArgs {
+    Views w;
+    const void *q;
+    const void *k;
+    const void *v;
+    const float *g;
+    const float *beta;
+    float *o;
+    int n_buf;         // tokens buffered before this one (windowed mode)
+};
+
+// d = d_k = d_v in {64, 128}; gate: LQ_GATE_*; in_dtype: LQ_DTYPE_*.
+cudaError_t launch_encode(const EncodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
+cudaError_t launch_decode_window(const DecodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
+cudaError_t launch_decode_fp32(const DecodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
+cudaError_t launch_decode_naive(const DecodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
+
+}  // namespace lq

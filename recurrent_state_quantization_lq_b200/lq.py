@@ -1,0 +1,230 @@
+"""Thin Python binding of liblq (include/lq.h): argument marshalling only.
+
+Every step of the decode path runs in liblq's CUDA kernels; PyTorch supplies
+device memory (the workspace and the input/output tensors) and streams.  If
+liblq.so has not been built, importing the library raises: there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblq.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "lq.h")
+
+# enums of include/lq.h
+LQ_OK, LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_WORKSPACE, LQ_ERR_WINDOW_FULL = 0, 1, 2, 3, 4
+LQ_ERR_RANGE, LQ_ERR_CUDA, LQ_ERR_DEVICE, LQ_ERR_STATE = 5, 6, 7, 8
+GATE = {"scalar": 0, "gdn": 0, "channel": 1, "kda": 1}
+MODE = {"window": 0, "naive": 1, "fp32": 2}
+SELECT = {"l2": 0, "maxabs": 1}
+DTYPE = {torch.float32: 0, torch.bfloat16: 1}
+ABSENT = ctypes.c_size_t(-1).value
+
+STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED", 3: "LQ_ERR_WORKSPACE",
+                4: "LQ_ERR_WINDOW_FULL", 5: "LQ_ERR_RANGE", 6: "LQ_ERR_CUDA", 7: "LQ_ERR_DEVICE",
+                8: "LQ_ERR_STATE"}
+
+
+class Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "heads", "d_k", "d_v", "window", "n_comp_rows", "n_comp_cols", "gate", "mode",
+        "smooth", "select", "in_dtype")]
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "total_bytes", "err", "codes", "row_scale", "col_smooth", "comp_index", "comp_row_vec",
+        "comp_col_vec", "gate_sum", "buf_delta", "buf_key", "buf_gate", "state_f32")] + \
+        [("comp_index_stride", ctypes.c_int32), ("window_pad", ctypes.c_int32)]
+
+
+class LQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}: {last_error()}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load liblq.so (built in-tree by ``python -m recurrent_state_quantization_lq_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m recurrent_state_quantization_lq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32 = ctypes.c_void_p, ctypes.c_int32
+        L.lq_workspace_bytes.argtypes = [ctypes.POINTER(Config)]
+        L.lq_workspace_bytes.restype = ctypes.c_size_t
+        L.lq_workspace_layout.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(Layout)]
+        L.lq_workspace_layout.restype = i32
+        L.lq_state_create.argtypes = [ctypes.POINTER(Config), vp, ctypes.c_size_t, ctypes.POINTER(vp)]
+        L.lq_state_create.restype = i32
+        L.lq_prefill_state.argtypes = [vp, vp, vp]
+        L.lq_prefill_state.restype = i32
+        L.lq_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
+        L.lq_decode_step.restype = i32
+        L.lq_window_flush.argtypes = [vp, vp]
+        L.lq_window_flush.restype = i32
+        L.lq_window_fill.argtypes = [vp]
+        L.lq_window_fill.restype = i32
+        L.lq_device_status.argtypes = [vp, vp]
+        L.lq_device_status.restype = i32
+        L.lq_state_destroy.argtypes = [vp]
+        L.lq_state_destroy.restype = i32
+        L.lq_last_error_string.argtypes = []
+        L.lq_last_error_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def header_symbols() -> list[str]:
+    """Names of the entry points include/lq.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"LQ_API\s+[\w\s\*]+?\b(lq_\w+)\s*\(", text)
+
+
+def last_error() -> str:
+    return lib().lq_last_error_string().decode()
+
+
+def make_config(batch: int, heads: int, d: int, window: int = 64, n_comp_rows: int = 2,
+                n_comp_cols: int = 2, gate: str = "scalar", mode: str = "window", smooth: int = 1,
+                select: str = "l2", in_dtype: torch.dtype = torch.bfloat16) -> Config:
+    return Config(batch, heads, d, d, window, n_comp_rows, n_comp_cols, GATE[gate], MODE[mode],
+                  smooth, SELECT[select], DTYPE[in_dtype])
+
+
+def workspace_bytes(cfg: Config) -> int:
+    return lib().lq_workspace_bytes(ctypes.byref(cfg))
+
+
+def workspace_layout(cfg: Config) -> Layout:
+    L = Layout()
+    st = lib().lq_workspace_layout(ctypes.byref(cfg), ctypes.byref(L))
+    if st != LQ_OK:
+        raise LQError(st, "lq_workspace_layout")
+    return L
+
+
+def _stream_ptr(stream, device) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(None if t is None else t.data_ptr())
+
+
+class DecodeState:
+    """A batch of (sequence, head) recurrent states of one layer, held by liblq.
+
+    The workspace is a torch uint8 tensor on ``device``; its regions can be
+    viewed with :meth:`view`.  All calls enqueue on ``stream`` (default: the
+    current stream) and return without synchronizing.
+    """
+
+    def __init__(self, batch: int, heads: int, d: int, *, window: int = 64, n_comp_rows: int = 2,
+                 n_comp_cols: int = 2, gate: str = "scalar", mode: str = "window", smooth: int = 1,
+                 select: str = "l2", in_dtype: torch.dtype = torch.bfloat16, device=None):
+        self.cfg = make_config(batch, heads, d, window, n_comp_rows, n_comp_cols, gate, mode, smooth,
+                               select, in_dtype)
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        nbytes = workspace_bytes(self.cfg)
+        if nbytes == 0:
+            raise LQError(LQ_ERR_INVALID_ARG, "lq_workspace_bytes")
+        self.layout = workspace_layout(self.cfg)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        h = ctypes.c_void_p()
+        st = lib().lq_state_create(ctypes.byref(self.cfg), _ptr(self.workspace), nbytes, ctypes.byref(h))
+        if st != LQ_OK:
+            raise LQError(st, "lq_state_create")
+        self._h = h
+        self.batch, self.heads, self.d = batch, heads, d
+        self.in_dtype = in_dtype
+        self.per_channel_gate = GATE[gate] == 1
+
+    # ------------------------------------------------------------------ calls
+    def _check(self, st: int, what: str) -> None:
+        if st != LQ_OK:
+            raise LQError(st, what)
+
+    def prefill(self, S0: torch.Tensor | None = None, stream=None) -> None:
+        if S0 is not None:
+            assert S0.dtype == torch.float32 and S0.is_contiguous() and S0.device == self.device
+            assert S0.numel() == self.batch * self.heads * self.d * self.d
+        self._check(lib().lq_prefill_state(self._h, _ptr(S0), _stream_ptr(stream, self.device)),
+                    "lq_prefill_state")
+
+    def decode_step(self, q, k, v, g, beta, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        if out is None:
+            out = torch.empty(self.batch, self.heads, self.d, dtype=torch.float32, device=self.device)
+        for t, dt in ((q, self.in_dtype), (k, self.in_dtype), (v, self.in_dtype), (g, torch.float32),
+                      (beta, torch.float32), (out, torch.float32)):
+            assert t.dtype == dt and t.is_contiguous() and t.device == self.device, (t.dtype, t.device)
+        self._check(lib().lq_decode_step(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(out),
+                                         _stream_ptr(stream, self.device)), "lq_decode_step")
+        return out
+
+    def flush(self, stream=None) -> None:
+        self._check(lib().lq_window_flush(self._h, _stream_ptr(stream, self.device)), "lq_window_flush")
+
+    @property
+    def fill(self) -> int:
+        return lib().lq_window_fill(self._h)
+
+    def device_status(self, stream=None) -> int:
+        """Synchronize and return the status of the device error word (LQ_OK if clean)."""
+        return lib().lq_device_status(self._h, _stream_ptr(stream, self.device))
+
+    # ------------------------------------------------------------ inspection
+    def view(self, name: str) -> torch.Tensor | None:
+        """A tensor view of one workspace region (see lq_layout in include/lq.h)."""
+        L, c = self.layout, self.cfg
+        off = getattr(L, name)
+        if off == ABSENT:
+            return None
+        N, d = c.batch * c.heads, c.d_k
+        gd = d if c.gate == 1 else 1
+        key_dt = torch.float32 if (c.gate == 1 or c.in_dtype == 0) else torch.bfloat16
+        nc = L.comp_index_stride
+        spec = {
+            "err": (torch.int32, (64,)),
+            "codes": (torch.int8, (c.batch, c.heads, d, d)),
+            "row_scale": (torch.float32, (c.batch, c.heads, d)),
+            "col_smooth": (torch.float32, (c.batch, c.heads, d)),
+            "comp_index": (torch.int32, (c.batch, c.heads, nc)),
+            "comp_row_vec": (torch.float32, (c.batch, c.heads, c.n_comp_rows, d)),
+            "comp_col_vec": (torch.float32, (c.batch, c.heads, c.n_comp_cols, d)),
+            "gate_sum": (torch.float64, (c.batch, c.heads, gd)),
+            "buf_delta": (torch.float32, (c.batch, c.heads, c.window, d)),
+            "buf_key": (key_dt, (c.batch, c.heads, c.window, d)),
+            "buf_gate": (torch.float64, (c.batch, c.heads, L.window_pad)),
+            "state_f32": (torch.float32, (c.batch, c.heads, d, d)),
+        }[name]
+        dt, shape = spec
+        n = 1
+        for s in shape:
+            n *= s
+        nbytes = n * torch.empty((), dtype=dt).element_size()
+        return self.workspace[off:off + nbytes].view(dt).view(shape)
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            lib().lq_state_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

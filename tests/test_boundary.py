@@ -1,0 +1,103 @@
+"""The C-ABI boundary without a GPU: the library loads, exports every entry
+point include/lq.h declares, validates configs and lays out workspaces.
+No call here launches a kernel."""
+import ctypes
+
+import pytest
+
+from recurrent_state_quantization_lq_b200 import lq
+
+
+def test_exports_every_declared_symbol():
+    names = lq.header_symbols()
+    assert set(names) >= {"lq_workspace_bytes", "lq_workspace_layout", "lq_state_create",
+                          "lq_prefill_state", "lq_decode_step", "lq_window_flush", "lq_window_fill",
+                          "lq_device_status", "lq_state_destroy", "lq_last_error_string"}
+    L = lq.lib()
+    for n in names:
+        assert hasattr(L, n), n
+
+
+@pytest.mark.parametrize("mode", ["window", "naive", "fp32"])
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_layout_regions_disjoint_aligned(mode, gate, d):
+    cfg = lq.make_config(3, 5, d, window=37, n_comp_rows=3, n_comp_cols=1, gate=gate, mode=mode)
+    L = lq.workspace_layout(cfg)
+    assert L.total_bytes == lq.workspace_bytes(cfg) > 0
+    N = 15
+    key_b = 4 if gate == "channel" else 2
+    sizes = {"err": 256, "codes": N * d * d, "row_scale": N * d * 4, "col_smooth": N * d * 4,
+             "comp_index": N * L.comp_index_stride * 4, "comp_row_vec": N * 3 * d * 4,
+             "comp_col_vec": N * 1 * d * 4, "gate_sum": N * (d if gate == "channel" else 1) * 8,
+             "buf_delta": N * 37 * d * 4, "buf_key": N * 37 * d * key_b,
+             "buf_gate": N * L.window_pad * 8, "state_f32": N * d * d * 4}
+    present = {
+        "window": {"err", "codes", "row_scale", "col_smooth", "comp_index", "comp_row_vec", "comp_col_vec",
+                   "gate_sum", "buf_delta", "buf_key"} | ({"buf_gate"} if gate == "scalar" else set()),
+        "naive": {"err", "codes", "row_scale"},
+        "fp32": {"err", "state_f32"},
+    }[mode]
+    spans = []
+    for name, size in sizes.items():
+        off = getattr(L, name)
+        if name in present:
+            assert off != lq.ABSENT and off % 256 == 0 and off + size <= L.total_bytes, name
+            spans.append((off, off + size))
+        else:
+            assert off == lq.ABSENT, name
+    spans.sort()
+    for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+        assert a1 <= b0
+    if mode == "window":
+        assert L.comp_index_stride == 4 and L.window_pad == 38
+
+
+@pytest.mark.parametrize("field,value", [("d_k", 96), ("d_v", 64), ("window", 0), ("window", 5000),
+                                         ("n_comp_rows", 17), ("n_comp_cols", -1), ("gate", 2),
+                                         ("mode", 3), ("smooth", 2), ("select", 2), ("in_dtype", 3),
+                                         ("batch", 0), ("heads", 0)])
+def test_invalid_configs_rejected(field, value):
+    cfg = lq.make_config(2, 2, 128)
+    setattr(cfg, field, value)
+    assert lq.workspace_bytes(cfg) == 0
+    assert lq.last_error() != ""
+    L = lq.Layout()
+    assert lq.lib().lq_workspace_layout(ctypes.byref(cfg), ctypes.byref(L)) == lq.LQ_ERR_INVALID_ARG
+
+
+def test_create_checks_workspace_and_lifecycle():
+    L = lq.lib()
+    cfg = lq.make_config(2, 2, 64, window=8)
+    need = lq.workspace_bytes(cfg)
+    h = ctypes.c_void_p()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: create is host-only
+    assert L.lq_state_create(ctypes.byref(cfg), None, need, ctypes.byref(h)) == lq.LQ_ERR_WORKSPACE
+    assert L.lq_state_create(ctypes.byref(cfg), ctypes.c_void_p((1 << 20) + 16), need,
+                             ctypes.byref(h)) == lq.LQ_ERR_WORKSPACE
+    assert L.lq_state_create(ctypes.byref(cfg), fake, need - 1, ctypes.byref(h)) == lq.LQ_ERR_WORKSPACE
+    assert "needs" in lq.last_error()
+    assert L.lq_state_create(ctypes.byref(cfg), fake, need, ctypes.byref(h)) == lq.LQ_OK
+    assert L.lq_window_fill(h) == 0
+    # decode and flush before prefill are refused on the host, before any launch
+    p = ctypes.c_void_p(1 << 21)
+    assert L.lq_decode_step(h, p, p, p, p, p, p, None) == lq.LQ_ERR_STATE
+    assert L.lq_window_flush(h, None) == lq.LQ_ERR_STATE
+    # null and misaligned inputs
+    assert L.lq_decode_step(h, None, p, p, p, p, p, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_decode_step(h, ctypes.c_void_p((1 << 21) + 8), p, p, p, p, p, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_state_destroy(h) == lq.LQ_OK
+    assert L.lq_window_fill(None) == -1
+    assert L.lq_state_destroy(None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_prefill_state(None, None, None) == lq.LQ_ERR_INVALID_ARG
+
+
+def test_flush_is_noop_outside_windowed_mode():
+    L = lq.lib()
+    for mode in ("naive", "fp32"):
+        cfg = lq.make_config(1, 1, 64, mode=mode)
+        h = ctypes.c_void_p()
+        assert L.lq_state_create(ctypes.byref(cfg), ctypes.c_void_p(1 << 20), lq.workspace_bytes(cfg),
+                                 ctypes.byref(h)) == lq.LQ_OK
+        assert L.lq_window_flush(h, None) == lq.LQ_OK
+        L.lq_state_destroy(h)

@@ -6,8 +6,8 @@ G_t = sum of the log-gates since the window start and gamma_t = exp(G_t):
   kappa_j = k_j / gamma_j,  delta_j = beta_j (v_j - S_{j-1}(alpha_j * k_j)),
 so a decode step needs only one pass over the fixed INT8 state plus the
 buffered (delta_j, kappa_j) pairs; compensators are buffered pairs with G = 0
-("Compensator Tokens, which share the update path of real tokens", LeapQuant,
-"Abstract (arXiv)").  The WY form writes the same product of transitions as
+(LeapQuant, "Abstract (arXiv)": Compensator Tokens take the same update path
+as real tokens).  The WY form writes the same product of transitions as
 Gamma_t - sum_j w_j (k_j * gamma_t / gamma_j)^T, and delta_t = v~_t - S~ u_t.
 These are checked against the oracle's dense recurrence and against explicit
 products of the transition matrices.
