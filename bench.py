@@ -1,0 +1,529 @@
+#!/usr/bin/env python
+"""Decode throughput of windowed INT8 GDN decode on B200, with its comparators.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one window of the workload for every one of L rotated layer-states:
+W decode launches per layer (one token for all 64 x 32 (sequence, head) units
+per launch) followed by one window flush per layer.  The L layer-states (4 by
+default, ~540 MB together) are visited round-robin like the layers of a model,
+so no layer's state is still in the 126 MB L2 when it is read again; L2 is not
+flushed.  value = decode tokens/s per layer = batch x W x L / step time.
+
+Also reported: the FP32-state and naive per-token INT8 decode kernels on the
+same inputs, the roofline of the dominant kernel (windowed decode, algorithmic
+bytes / event-timed duration vs the measured HBM copy bandwidth), an
+end-to-end number through the public API with host buffers, the oracle on the
+host cores, and the SM clocks sampled during the timed region.
+
+Under torchrun each rank runs its own batch of sequences (independent units,
+no collective on the data path); rank 0 prints the JSON line with the
+whole-job value, timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from recurrent_state_quantization_lq_b200 import inputs  # noqa: E402
+
+METRIC = "decode tokens/s per layer & achieved HBM GB/s vs 8 TB/s roofline (INT8 vs FP32 state)"
+UNIT = "tokens/s per layer"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------ byte accounting
+
+def decode_window_bytes(d: int, in_b: int, kda: bool, ncr: int, ncc: int, n_buf: int) -> int:
+    """Algorithmic HBM bytes one (sequence, head) unit moves in one windowed
+    decode step with n_buf tokens buffered."""
+    cis = ((ncr + ncc + 3) // 4) * 4
+    fixed = d * d + 4 * d + 4 * d            # INT8 tile, row scales, smoothing factors
+    fixed += 3 * in_b * d + 4                # q, k, v, beta
+    fixed += 4 * cis + 4 * d * (ncr + ncc)   # compensators
+    fixed += 4 * d + 4 * d                   # o written, delta_t appended
+    if kda:
+        fixed += 4 * d + 8 * d + 8 * d       # g read, G read + written
+        fixed += 4 * d                       # kappa_t appended
+        per_entry = 4 * d + 4 * d            # delta_j, kappa_j
+    else:
+        fixed += 4 + 8 + 8 + 8               # g read, G read + written, G_t appended
+        fixed += in_b * d                    # k_t appended
+        per_entry = 4 * d + in_b * d + 8     # delta_j, k_j, G_j
+    return fixed + per_entry * n_buf
+
+
+def flush_bytes(d: int, in_b: int, kda: bool, ncr: int, ncc: int, n_buf: int) -> int:
+    """Algorithmic bytes of one unit's window flush (read the window-start state
+    and the buffer, write the new state)."""
+    cis = ((ncr + ncc + 3) // 4) * 4
+    state = d * d + 8 * d + 4 * cis + 4 * d * (ncr + ncc)
+    gd = d if kda else 1
+    entry = 4 * d + (4 * d if kda else in_b * d + 8)
+    return 2 * state + 2 * 8 * gd + entry * n_buf
+
+
+def fp32_bytes(d: int, in_b: int, kda: bool) -> int:
+    return 8 * d * d + 3 * in_b * d + 4 + (4 * d if kda else 4) + 4 * d
+
+
+def naive_bytes(d: int, in_b: int, kda: bool) -> int:
+    return 2 * (d * d + 4 * d) + 3 * in_b * d + 4 + (4 * d if kda else 4) + 4 * d
+
+
+# --------------------------------------------------------------- environment
+
+def measured_hbm_gbs() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        try:
+            p = torch.cuda.get_device_properties(device_index)
+            self.gpu = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        except Exception:
+            self.gpu = str(device_index)
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# -------------------------------------------------------------- distributed
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ the CPU oracle
+
+def oracle_sample(wl: inputs.Workload, n_units: int, n_tokens: int, n_threads: int, seed: int) -> tuple[float, int]:
+    """Time the oracle's windowed decode on a sample of units; returns
+    (seconds, threads used)."""
+    import numpy as np
+
+    import oracle
+    d = wl.d_k
+    gate = oracle.GATE_CHANNEL if wl.per_channel_gate else oracle.GATE_SCALAR
+    p = oracle.Params(d, d, window=wl.window, n_comp_rows=wl.n_comp_rows, n_comp_cols=wl.n_comp_cols,
+                      gate=gate, mode=oracle.MODE_WINDOW)
+    tb = inputs.tokens(seed, 0, n_tokens, 1, n_units, d, d, wl.per_channel_gate, wl.dtype)
+
+    def heads(x):
+        return x.reshape(n_tokens, n_units, *x.shape[3:]).transpose(0, 1).double().numpy()
+
+    S0 = 0.1 * torch.randn(n_units, d, d, generator=torch.Generator().manual_seed(seed)).double().numpy()
+    args = (heads(tb.q), heads(tb.k), heads(tb.v), heads(tb.g), heads(tb.beta))
+    used = oracle.max_threads(n_threads)
+    t0 = time.perf_counter()
+    oracle.run(p, S0, *args, snapshots=False, n_threads=n_threads)
+    return time.perf_counter() - t0, used
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ our arm
+
+class LayerStack:
+    """L independent layer-states of one workload, their token inputs and
+    CUDA graphs of each window (decode launches, then flushes)."""
+
+    def __init__(self, wl, n_layers, mode, device, seed, tokens_per_layer, prefill_states=None):
+        from recurrent_state_quantization_lq_b200 import lq
+        gate = "channel" if wl.per_channel_gate else "scalar"
+        self.wl, self.mode, self.L = wl, mode, n_layers
+        self.states = [lq.DecodeState(wl.batch, wl.heads, wl.d_k, window=wl.window,
+                                      n_comp_rows=wl.n_comp_rows, n_comp_cols=wl.n_comp_cols, gate=gate,
+                                      mode=mode, in_dtype=wl.dtype, device=device) for _ in range(n_layers)]
+        self.tok = [inputs.tokens_on_device(seed * 100 + l, tokens_per_layer, wl.batch, wl.heads, wl.d_k,
+                                            wl.d_v, wl.per_channel_gate, wl.dtype, device)
+                    for l in range(n_layers)]
+        self.out = torch.empty(n_layers, wl.batch, wl.heads, wl.d_v, dtype=torch.float32, device=device)
+        for l, st in enumerate(self.states):
+            st.prefill(prefill_states[l] if prefill_states is not None else None)
+        self.T = tokens_per_layer
+
+    def decode(self, l, t):
+        tb = self.tok[l]
+        self.states[l].decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=self.out[l])
+
+    def capture(self, window_index, stream):
+        """Two graphs for one window: W x L decode launches, then L flushes."""
+        W = self.wl.window
+        gd, gf = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd, stream=stream):
+            for i in range(W):
+                t = (window_index * W + i) % self.T
+                for l in range(self.L):
+                    self.decode(l, t)
+        with torch.cuda.graph(gf, stream=stream):
+            for st in self.states:
+                st.flush()
+        return gd, gf
+
+
+def fp32_prefill(wl, n_layers, device, seed):
+    """Per layer: the FP32 recurrence over the workload's prefill tokens from zero."""
+    from recurrent_state_quantization_lq_b200 import lq
+    gate = "channel" if wl.per_channel_gate else "scalar"
+    S = []
+    for l in range(n_layers):
+        st = lq.DecodeState(wl.batch, wl.heads, wl.d_k, gate=gate, mode="fp32", in_dtype=wl.dtype, device=device)
+        st.prefill(None)
+        tb = inputs.tokens_on_device(seed * 100 + 50 + l, wl.prefill_tokens, wl.batch, wl.heads, wl.d_k, wl.d_v,
+                                     wl.per_channel_gate, wl.dtype, device)
+        for t in range(wl.prefill_tokens):
+            st.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t])
+        S.append(st.view("state_f32").clone())
+        del st, tb
+    torch.cuda.synchronize()
+    return S
+
+
+def run_ours(args, rank, world, local):
+    from recurrent_state_quantization_lq_b200 import lq
+    dev = torch.device("cuda", local)
+    wl = inputs.WORKLOADS[args.workload]
+    L, W, K, WU = args.layers, wl.window, args.steps, args.warmup
+    d, kda = wl.d_k, wl.per_channel_gate
+    in_b = 2 if wl.dtype == torch.bfloat16 else 4
+    ncr, ncc = wl.n_comp_rows, wl.n_comp_cols
+    seed = wl.seed * 1000 + rank
+    stream = torch.cuda.Stream(device=dev)
+    n_windows = max(1, wl.decode_tokens // W)
+
+    S0 = fp32_prefill(wl, L, dev, seed)
+    win = LayerStack(wl, L, "window", dev, seed, wl.decode_tokens, S0)
+    # warm-up launches outside capture (sets kernel attributes)
+    with torch.cuda.stream(stream):
+        for l in range(L):
+            win.decode(l, 0)
+            win.states[l].flush()
+    torch.cuda.synchronize()
+    graphs = []
+    for wi in range(n_windows):
+        graphs.append(win.capture(wi, stream))
+    torch.cuda.synchronize()
+
+    def run_steps(n, first, evs=None):
+        with torch.cuda.stream(stream):
+            for s in range(n):
+                gd, gf = graphs[(first + s) % n_windows]
+                if evs is not None:
+                    evs[s][0].record(stream)
+                gd.replay()
+                if evs is not None:
+                    evs[s][1].record(stream)
+                gf.replay()
+                if evs is not None:
+                    evs[s][2].record(stream)
+
+    run_steps(WU, 0)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        run_steps(K, WU, evs)
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = max_over_ranks(start.elapsed_time(end), world)
+    ms_step = ms_total / K
+    dec_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    fl_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    for st in win.states:
+        assert st.device_status(stream) == lq.LQ_OK, lq.last_error()
+
+    units = wl.batch * wl.heads
+    # algorithmic bytes of all decode launches and flushes in the timed region
+    dec_bytes = K * L * units * sum(decode_window_bytes(d, in_b, kda, ncr, ncc, n) for n in range(W))
+    fl_bytes = K * L * units * flush_bytes(d, in_b, kda, ncr, ncc, W)
+    n_dec = K * L * W
+    dec_avg_us = dec_ms * 1e3 / n_dec
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_gbs()
+    # weak scaling: the job's tokens are every rank's tokens over the slowest rank's time
+    value = world * wl.batch * W * L * K / (ms_total * 1e-3)
+
+    # ---- comparators on the same workload (same inputs recipe, same rotation)
+    comps = {}
+    Kc = max(4, min(K, args.comparator_steps))
+    for mode, nbytes in (("fp32", fp32_bytes(d, in_b, kda)), ("naive", naive_bytes(d, in_b, kda))):
+        stk = LayerStack(wl, L, mode, dev, seed, W, S0)
+        with torch.cuda.stream(stream):
+            for l in range(L):
+                stk.decode(l, 0)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(W):
+                for l in range(L):
+                    stk.decode(l, i)
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(Kc):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1), world) / Kc
+        comps[mode] = {"value": world * wl.batch * W * L / (ms * 1e-3), "ms_per_step": ms,
+                       "hbm_gbs": units * nbytes * W * L / (ms * 1e-3) / 1e9,
+                       "bytes_per_unit_token": nbytes}
+        del g, stk
+        torch.cuda.synchronize()
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Ke = max(2, min(K, args.e2e_steps))
+        tb0 = [inputs.TokenBatch(*(x[:W].cpu().pin_memory() for x in (tb.q, tb.k, tb.v, tb.g, tb.beta)))
+               for tb in win.tok]
+        dev_in = [inputs.TokenBatch(*(torch.empty_like(x, device=dev) for x in (tb.q, tb.k, tb.v, tb.g, tb.beta)))
+                  for tb in tb0]
+        out_dev = torch.empty(L, W, wl.batch, wl.heads, wl.d_v, dtype=torch.float32, device=dev)
+        out_host = torch.empty(out_dev.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for tb in tb0 for x in (tb.q, tb.k, tb.v, tb.g, tb.beta))
+        d2h = out_host.numel() * 4
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for l in range(L):
+                    for src, dst in zip((tb0[l].q, tb0[l].k, tb0[l].v, tb0[l].g, tb0[l].beta),
+                                        (dev_in[l].q, dev_in[l].k, dev_in[l].v, dev_in[l].g, dev_in[l].beta)):
+                        dst.copy_(src, non_blocking=True)
+                for i in range(W):
+                    for l in range(L):
+                        b = dev_in[l]
+                        win.states[l].decode_step(b.q[i], b.k[i], b.v[i], b.g[i], b.beta[i], out=out_dev[l, i],
+                                                  stream=stream)
+                for st in win.states:
+                    st.flush(stream=stream)
+                out_host.copy_(out_dev, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1), world) / Ke
+        e2e = {"value": world * wl.batch * W * L / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "path": "DecodeState.decode_step/flush (C ABI), pinned host inputs copied in and outputs copied out each step"}
+
+    # ---- the oracle on the host cores (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = host_cores()
+        n_units = min(units, 8 * threads)
+        n_tok = args.cpu_tokens
+        secs, used = oracle_sample(wl, n_units, n_tok, threads, seed)
+        cpu = {"value": n_units * n_tok / wl.heads / secs, "unit": UNIT, "cores": used, "kind": "oracle",
+               "sample": f"{n_units} (sequence, head) units x {n_tok} decode tokens of {wl.name} "
+                         f"(windowed mode, W={W}, dense FP64 recurrence), {secs:.1f} s"}
+
+    clocks = clk.summary()
+    roofline = {"bound": "hbm", "kernel": "decode_window_kernel", "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s", "traffic": None,
+                "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS,
+                "avg_launch_us": dec_avg_us, "bytes_per_launch": dec_bytes / n_dec}
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": WU,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
+                   "heads": wl.heads, "d_k": d, "d_v": d, "window": W, "n_comp": ncr + ncc,
+                   "gate": "per-key-channel (KDA)" if kda else "scalar (GDN)", "state": "int8 + fp32 buffer",
+                   "inputs": "bf16 q/k/v, fp32 g/beta" if in_b == 2 else "fp32",
+                   "layers_rotated": L,
+                   "step": f"one window per layer: {W} decode launches + 1 flush, x{L} layers",
+                   "l2": f"not flushed; {L} layer-states rotated, working set > L2",
+                   "parallelism": f"dp{world} (independent sequences per GPU, no collective)"},
+        "hbm_gbs": achieved,
+        "decode_ms_per_step": dec_ms / K, "flush_ms_per_step": fl_ms / K,
+        "flush_gbs": fl_bytes / (fl_ms * 1e-3) / 1e9,
+        "fp32_state": comps["fp32"], "naive_int8": comps["naive"],
+        "speedup_vs_fp32_state": value / comps["fp32"]["value"],
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": K * L * (W + 1), "clocks": clocks,
+    }
+    return res
+
+
+# ------------------------------------------------------------ reference arm
+
+def run_reference(args, rank, world):
+    """The oracle, as it stands, on the host cores: the reference arm."""
+    if rank != 0:
+        return None
+    wl = inputs.WORKLOADS[args.workload]
+    threads = host_cores()
+    n_units = min(wl.units, 2 * threads)
+    n_tok = 16
+    for _ in range(args.warmup):
+        oracle_sample(wl, n_units, n_tok, threads, 7)
+    total, used = 0.0, 1
+    for s in range(args.steps):
+        secs, used = oracle_sample(wl, n_units, n_tok, threads, 11 + s)
+        total += secs
+    ms = total / args.steps * 1e3
+    value = n_units * n_tok / wl.heads / (ms * 1e-3)
+    sample = (f"{n_units} (sequence, head) units x {n_tok} decode tokens of {wl.name} per step "
+              f"(windowed mode, dense FP64 recurrence)")
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "heads": wl.heads, "d_k": wl.d_k,
+                       "window": wl.window, "n_comp": wl.n_comp_rows + wl.n_comp_cols},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=240)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gdn_b64_h32_d128_w64", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--layers", type=int, default=4)
+    ap.add_argument("--comparator-steps", type=int, default=40)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-tokens", type=int, default=192)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        res = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

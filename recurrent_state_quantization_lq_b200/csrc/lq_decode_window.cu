@@ -380,9 +380,18 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
     using Sh = DecShape<D, KDA, InT, KeyT>;
     const DecLayout L = Sh::layout(a.w.n_comp_rows, a.w.n_comp_cols, a.w.comp_index_stride);
     auto kern = decode_window_kernel<D, KDA, InT, KeyT>;
+    // The opt-in shared-memory size is set once per device and size, so that
+    // launches inside a stream capture make no attribute calls.
+    static int opted_in[64] = {0};
     if (L.total > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= 64 || opted_in[dev] < L.total) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < 64) opted_in[dev] = L.total;
+        }
     }
     kern<<<a.w.units, kThreads, L.total, s>>>(a);
     return cudaGetLastError();

@@ -141,3 +141,29 @@ def sweep_workload(batch: int, window: int) -> Workload:
     """One point of the GDN batch x window sweep (32 heads, 128x128, 2048 tokens, n_c=4)."""
     return Workload(f"gdn_sweep_b{batch}_w{window}", batch, 32, 128, 128, window, 2, 2, False,
                     512, 2048, torch.bfloat16, 4)
+
+
+def tokens_on_device(seed: int, T: int, batch: int, heads: int, d_k: int, d_v: int,
+                     per_channel_gate: bool, dtype: torch.dtype, device,
+                     chunk: int = 64) -> TokenBatch:
+    """The same recipe drawn on the GPU from a CUDA generator (for timing runs
+    that need gigabytes of tokens; its stream differs from `tokens`)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed * _TOKEN_MIX + 17)
+    q = torch.empty(T, batch, heads, d_k, dtype=dtype, device=device)
+    k = torch.empty_like(q)
+    v = torch.empty(T, batch, heads, d_v, dtype=dtype, device=device)
+    gshape = (batch, heads, d_k) if per_channel_gate else (batch, heads)
+    g = torch.empty((T,) + gshape, dtype=torch.float32, device=device)
+    beta = torch.empty(T, batch, heads, dtype=torch.float32, device=device)
+    for t0 in range(0, T, chunk):
+        n = min(chunk, T - t0)
+        x = torch.randn(n, batch, heads, d_k, generator=gen, device=device)
+        q[t0:t0 + n] = (x / x.norm(dim=-1, keepdim=True)).to(dtype)
+        x = torch.randn(n, batch, heads, d_k, generator=gen, device=device)
+        k[t0:t0 + n] = (x / x.norm(dim=-1, keepdim=True)).to(dtype)
+        v[t0:t0 + n] = torch.randn(n, batch, heads, d_v, generator=gen, device=device).to(dtype)
+        beta[t0:t0 + n] = torch.sigmoid(torch.randn(n, batch, heads, generator=gen, device=device))
+        g[t0:t0 + n] = -0.1 * torch.nn.functional.softplus(
+            torch.randn((n,) + gshape, generator=gen, device=device))
+    return TokenBatch(q, k, v, g, beta)

@@ -138,7 +138,10 @@ class DecodeState:
                  select: str = "l2", in_dtype: torch.dtype = torch.bfloat16, device=None):
         self.cfg = make_config(batch, heads, d, window, n_comp_rows, n_comp_cols, gate, mode, smooth,
                                select, in_dtype)
-        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        dev = torch.device(device) if device is not None else torch.device("cuda")
+        if dev.index is None:
+            dev = torch.device(dev.type, torch.cuda.current_device())
+        self.device = dev
         nbytes = workspace_bytes(self.cfg)
         if nbytes == 0:
             raise LQError(LQ_ERR_INVALID_ARG, "lq_workspace_bytes")
