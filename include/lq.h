@@ -91,8 +91,8 @@ typedef struct lq_config {
     int32_t d_k;          /* key channels: 64 or 128                             */
     int32_t d_v;          /* value channels: equal to d_k                        */
     int32_t window;       /* W, tokens per window, 1..4096 (windowed mode)       */
-    int32_t n_comp_rows;  /* compensator rows, 0..16 (windowed mode)             */
-    int32_t n_comp_cols;  /* compensator columns, 0..16 (windowed mode)          */
+    int32_t n_comp_rows;  /* compensator rows, 0..8 (windowed mode)              */
+    int32_t n_comp_cols;  /* compensator columns, 0..8 (windowed mode)           */
     int32_t gate;         /* LQ_GATE_SCALAR or LQ_GATE_CHANNEL                   */
     int32_t mode;         /* LQ_MODE_*                                           */
     int32_t smooth;       /* 1: column smoothing before quantization (windowed)  */

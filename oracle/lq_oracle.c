@@ -140,9 +140,11 @@ static int argmax_free(const float *score, const unsigned char *taken, int n)
  *     m_j = max_i |R_ij|, s_j = sqrt(m_j) rounded to FP32; reading: s_j = 1
  *     where m_j = 0.  Without smoothing s_j = 1.
  *  3. Per-row symmetric INT8 ([abs]: the state is held in 8 bits):
- *     R'_ij = R_ij / s_j, sigma_i = max_j |R'_ij| / 127,
- *     Q_ij = clamp(rint(R'_ij / sigma_i), -127, 127) with ties to even;
- *     reading: Q_i = 0 where sigma_i = 0.
+ *     R'_ij = R_ij * (1 / s_j), M_i = max_j |R'_ij|, sigma_i = M_i / 127,
+ *     Q_ij = clamp(rint(R'_ij * (127 / M_i)), -127, 127) with ties to even;
+ *     reading: Q_i = 0 where M_i = 0.  The scales are applied as
+ *     multiplications by FP32 reciprocals (one division per column and per
+ *     row); the pages fix no arithmetic for the quantizer.
  *  4. S~_ij = sigma_i Q_ij s_j + C_ij, C the sum of the compensator pairs.
  *
  * comp_idx: n_rows row indices then n_cols column indices.
@@ -156,6 +158,7 @@ void lqo_encode(const lqo_params *p, int n_rows, int n_cols, int smooth, int sel
     float *R = (float *)malloc(sizeof(float) * dv * dk);
     float *score = (float *)malloc(sizeof(float) * (dv > dk ? dv : dk));
     unsigned char *taken = (unsigned char *)calloc((size_t)(dv > dk ? dv : dk), 1);
+    float *rs = (float *)malloc(sizeof(float) * dk);
 
     for (int e = 0; e < dv * dk; ++e) R[e] = (float)S[e];
 
@@ -209,17 +212,19 @@ void lqo_encode(const lqo_params *p, int n_rows, int n_cols, int smooth, int sel
         s[j] = (smooth && m > 0.0f) ? sqrtf(m) : 1.0f;
     }
     /* 3. row scales and codes */
+    for (int j = 0; j < dk; ++j) rs[j] = 1.0f / s[j];
     for (int i = 0; i < dv; ++i) {
         float mx = 0.0f;
         for (int j = 0; j < dk; ++j) {
-            float a = fabsf(R[i * dk + j] / s[j]);
+            float a = fabsf(R[i * dk + j] * rs[j]);
             if (a > mx) mx = a;
         }
         sigma[i] = mx / 127.0f;
+        float rho = (mx > 0.0f) ? 127.0f / mx : 0.0f;
         for (int j = 0; j < dk; ++j) {
             float code = 0.0f;
-            if (sigma[i] > 0.0f) {
-                code = rintf((R[i * dk + j] / s[j]) / sigma[i]);
+            if (mx > 0.0f) {
+                code = rintf((R[i * dk + j] * rs[j]) * rho);
                 if (code > 127.0f) code = 127.0f;
                 if (code < -127.0f) code = -127.0f;
             }
@@ -241,6 +246,7 @@ void lqo_encode(const lqo_params *p, int n_rows, int n_cols, int smooth, int sel
     free(R);
     free(score);
     free(taken);
+    free(rs);
 }
 
 /* Number of codec applications in a run of T tokens: the prefill encoding,

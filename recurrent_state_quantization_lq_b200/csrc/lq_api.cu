@@ -18,7 +18,7 @@ lq_status fail(lq_status code, const std::string &why) {
 }
 
 constexpr uint32_t kMagic = 0x4c515354u;  // "LQST"
-constexpr int kMaxComp = 16;
+constexpr int kMaxComp = 8;
 constexpr int kMaxWindow = 4096;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -37,7 +37,7 @@ bool validate(const lq_config *c, std::string *why) {
     if (c->mode == LQ_MODE_WINDOW) {
         if (c->window < 1 || c->window > kMaxWindow) { *why = "window must be in 1..4096"; return false; }
         if (c->n_comp_rows < 0 || c->n_comp_rows > kMaxComp || c->n_comp_cols < 0 || c->n_comp_cols > kMaxComp) {
-            *why = "n_comp_rows and n_comp_cols must be in 0..16"; return false;
+            *why = "n_comp_rows and n_comp_cols must be in 0..8"; return false;
         }
         if (c->smooth != 0 && c->smooth != 1) { *why = "smooth must be 0 or 1"; return false; }
         if (c->select != LQ_SELECT_L2 && c->select != LQ_SELECT_MAXABS) { *why = "select must be LQ_SELECT_L2 or LQ_SELECT_MAXABS"; return false; }

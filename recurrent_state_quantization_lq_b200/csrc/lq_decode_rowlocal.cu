@@ -11,8 +11,8 @@
 // The FP32 kernel reads and writes the FP32 row.  The naive kernel
 // dequantizes the row (sigma_i Q_ij), applies the same update, emits o from
 // the updated FP32 row, then requantizes it with a fresh per-row scale
-// (sigma'_i = max_j |S'_ij| / 127, Q'_ij = rint(S'_ij / sigma'_i)) and no
-// compensators or smoothing.  One CTA per (sequence, head), rows spread over
+// (M_i = max_j |S'_ij|, sigma'_i = M_i / 127, Q'_ij = rint(S'_ij * (127 / M_i)))
+// and no compensators or smoothing.  One CTA per (sequence, head), rows spread over
 // lanes groups with 16-byte vector loads.
 #include "lq_kernels.h"
 
@@ -181,14 +181,14 @@ __global__ void __launch_bounds__(kThreads) decode_naive_kernel(DecodeArgs a) {
         po = group_sum<LPR>(po);
         m = group_max<LPR>(m);
         const float sigma = __fdiv_rn(m, 127.0f);
+        const float rho = (m > 0.0f) ? __fdiv_rn(127.0f, m) : 0.0f;
         uint32_t out[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
             uint32_t word = 0;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float code = 0.0f;
-                if (sigma > 0.0f) code = fminf(fmaxf(rintf(__fdiv_rn(R[4 * h + c], sigma)), -127.0f), 127.0f);
+                const float code = fminf(fmaxf(rintf(__fmul_rn(R[4 * h + c], rho)), -127.0f), 127.0f);
                 word |= (uint32_t)((int)code & 0xff) << (8 * c);
             }
             out[h] = word;

@@ -13,10 +13,12 @@
 //   2. compensator rows (largest L2 norm, or max-abs), then columns of the
 //      row-zeroed residual, stored as FP32 pairs and zeroed;
 //   3. s_j = sqrt(max_i |R_ij|) (1 for an empty column);
-//   4. sigma_i = max_j |R_ij / s_j| / 127, Q_ij = rint((R_ij / s_j) / sigma_i).
+//   4. R'_ij = R_ij * (1/s_j), M_i = max_j |R'_ij|, sigma_i = M_i / 127,
+//      Q_ij = rint(R'_ij * (127 / M_i)).
 // Every value that decides a code is computed with IEEE round-to-nearest FP32
-// division and square root, so a given FP32 state always encodes to the same
-// codes, scales and smoothing factors.
+// operations (square root, one division per column and per row, products
+// without fused adds), so a given FP32 state always encodes to the same codes,
+// scales and smoothing factors.
 #include "lq_kernels.h"
 
 namespace lq {
@@ -67,14 +69,17 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
     float *sh_part = sh_kap + kEncChunk * D;                    // [16][D]
     float *sh_gam = sh_part + 16 * D;                           // [D] gamma_W per key channel
     float *sh_score = sh_gam + D;                               // [D]
-    float *sh_s = sh_score + D;                                 // [D] smoothing factors
+    float *sh_s = sh_score + D;                                 // [D] 1 / smoothing factor
     float *sh_fac = sh_s + D;                                   // [chunk]
     int *sh_sel = reinterpret_cast<int *>(sh_fac + kEncChunk);  // [32]: rows then columns
 
     auto row_of = [&](int r) { return (r >> 2) * 64 + ty * 4 + (r & 3); };
     auto col_of = [&](int c) { return (c >> 2) * 64 + tx * 4 + (c & 3); };
 
-    float acc[NR][NR];
+    // The tile lives in registers as column pairs so the rank update can use
+    // packed FP32 FMAs; ACC(r, c) names one element.
+    float2 acc2[NR][NR / 2];
+#define ACC(r, c) ((((c) & 1) != 0) ? acc2[r][(c) >> 1].y : acc2[r][(c) >> 1].x)
 
     // ------------------------------------------------------------ 1. rebuild
     if (!a.from_buffer) {
@@ -85,14 +90,14 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     float4 x = *reinterpret_cast<const float4 *>(S0 + (size_t)row_of(r) * D + g * 64 + tx * 4);
-                    acc[r][g * 4 + 0] = x.x; acc[r][g * 4 + 1] = x.y;
-                    acc[r][g * 4 + 2] = x.z; acc[r][g * 4 + 3] = x.w;
+                    ACC(r, g * 4 + 0) = x.x; ACC(r, g * 4 + 1) = x.y;
+                    ACC(r, g * 4 + 2) = x.z; ACC(r, g * 4 + 3) = x.w;
                 }
         } else {
 #pragma unroll
             for (int r = 0; r < NR; ++r)
 #pragma unroll
-                for (int c = 0; c < NR; ++c) acc[r][c] = 0.0f;
+                for (int c = 0; c < NR; ++c) ACC(r, c) = 0.0f;
         }
     } else {
         // gamma_W per key channel (scalar gate: one value for all)
@@ -119,10 +124,10 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
                 uint32_t word = *reinterpret_cast<const uint32_t *>(Qu + (size_t)row_of(r) * D + g * 64 + tx * 4);
                 float f0, f1, f2, f3;
                 i8x4_to_f32(word, f0, f1, f2, f3);
-                acc[r][g * 4 + 0] = (si * f0) * sg[g * 4 + 0];
-                acc[r][g * 4 + 1] = (si * f1) * sg[g * 4 + 1];
-                acc[r][g * 4 + 2] = (si * f2) * sg[g * 4 + 2];
-                acc[r][g * 4 + 3] = (si * f3) * sg[g * 4 + 3];
+                ACC(r, g * 4 + 0) = (si * f0) * sg[g * 4 + 0];
+                ACC(r, g * 4 + 1) = (si * f1) * sg[g * 4 + 1];
+                ACC(r, g * 4 + 2) = (si * f2) * sg[g * 4 + 2];
+                ACC(r, g * 4 + 3) = (si * f3) * sg[g * 4 + 3];
             }
         }
         // compensators (entries with G = 0), then the buffered tokens
@@ -163,18 +168,22 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
             }
             __syncthreads();
             for (int el = 0; el < ne; ++el) {
-                float dr[NR], kc[NR];
+                float dr[NR];
+                float2 kc[NR / 2];
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     float4 x = *reinterpret_cast<const float4 *>(sh_delta + el * D + g * 64 + ty * 4);
                     float4 y = *reinterpret_cast<const float4 *>(sh_kap + el * D + g * 64 + tx * 4);
                     dr[g * 4 + 0] = x.x; dr[g * 4 + 1] = x.y; dr[g * 4 + 2] = x.z; dr[g * 4 + 3] = x.w;
-                    kc[g * 4 + 0] = y.x; kc[g * 4 + 1] = y.y; kc[g * 4 + 2] = y.z; kc[g * 4 + 3] = y.w;
+                    kc[g * 2 + 0] = make_float2(y.x, y.y);
+                    kc[g * 2 + 1] = make_float2(y.z, y.w);
                 }
 #pragma unroll
-                for (int r = 0; r < NR; ++r)
+                for (int r = 0; r < NR; ++r) {
+                    const float2 dd = make_float2(dr[r], dr[r]);
 #pragma unroll
-                    for (int c = 0; c < NR; ++c) acc[r][c] = fmaf(dr[r], kc[c], acc[r][c]);
+                    for (int m = 0; m < NR / 2; ++m) acc2[r][m] = __ffma2_rn(dd, kc[m], acc2[r][m]);
+                }
             }
             __syncthreads();
         }
@@ -187,7 +196,7 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
             float p = 0.0f;
 #pragma unroll
             for (int c = 0; c < NR; ++c) {
-                const float x = fabsf(acc[r][c]);
+                const float x = fabsf(ACC(r, c));
                 p = (a.select == LQ_SELECT_L2) ? p + x * x : fmaxf(p, x);
             }
             p = (a.select == LQ_SELECT_L2) ? group_sum<16>(p) : group_max<16>(p);
@@ -214,9 +223,9 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
 #pragma unroll
                     for (int g = 0; g < G; ++g)
                         *reinterpret_cast<float4 *>(dst + g * 64 + tx * 4) =
-                            make_float4(acc[r][g * 4], acc[r][g * 4 + 1], acc[r][g * 4 + 2], acc[r][g * 4 + 3]);
+                            make_float4(ACC(r, g * 4), ACC(r, g * 4 + 1), ACC(r, g * 4 + 2), ACC(r, g * 4 + 3));
 #pragma unroll
-                    for (int cc = 0; cc < NR; ++cc) acc[r][cc] = 0.0f;
+                    for (int cc = 0; cc < NR; ++cc) ACC(r, cc) = 0.0f;
                 }
             }
         }
@@ -229,7 +238,7 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
             float p = 0.0f;
 #pragma unroll
             for (int r = 0; r < NR; ++r) {
-                const float x = fabsf(acc[r][c]);
+                const float x = fabsf(ACC(r, c));
                 p = (a.select == LQ_SELECT_L2) ? p + x * x : fmaxf(p, x);
             }
             sh_part[ty * D + col_of(c)] = p;
@@ -264,9 +273,9 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
 #pragma unroll
                     for (int g = 0; g < G; ++g)
                         *reinterpret_cast<float4 *>(dst + g * 64 + ty * 4) =
-                            make_float4(acc[g * 4][c], acc[g * 4 + 1][c], acc[g * 4 + 2][c], acc[g * 4 + 3][c]);
+                            make_float4(ACC(g * 4, c), ACC(g * 4 + 1, c), ACC(g * 4 + 2, c), ACC(g * 4 + 3, c));
 #pragma unroll
-                    for (int r = 0; r < NR; ++r) acc[r][c] = 0.0f;
+                    for (int r = 0; r < NR; ++r) ACC(r, c) = 0.0f;
                 }
             }
         }
@@ -277,7 +286,7 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
     for (int c = 0; c < NR; ++c) {
         float m = 0.0f;
 #pragma unroll
-        for (int r = 0; r < NR; ++r) m = fmaxf(m, fabsf(acc[r][c]));
+        for (int r = 0; r < NR; ++r) m = fmaxf(m, fabsf(ACC(r, c)));
         sh_part[ty * D + col_of(c)] = m;
     }
     __syncthreads();
@@ -285,34 +294,36 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
         float m = 0.0f;
         for (int y = 0; y < 16; ++y) m = fmaxf(m, sh_part[y * D + j]);
         const float s = (a.smooth && m > 0.0f) ? __fsqrt_rn(m) : 1.0f;
-        sh_s[j] = s;
+        sh_s[j] = __fdiv_rn(1.0f, s);          // applied as a multiplication
         if (w.col_smooth != nullptr) w.col_smooth[(size_t)u * D + j] = s;
     }
     __syncthreads();
 
     // ------------------------------------------ 4. row scales and the codes
-    float sc[NR];
+    // R'_ij = R_ij * (1/s_j); M_i = max_j |R'_ij|; sigma_i = M_i / 127;
+    // Q_ij = rint(R'_ij * (127 / M_i)).
+    float rs[NR];
 #pragma unroll
-    for (int c = 0; c < NR; ++c) sc[c] = sh_s[col_of(c)];
+    for (int c = 0; c < NR; ++c) rs[c] = sh_s[col_of(c)];
     int8_t *Qu = w.codes + (size_t)u * D * D;
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
         float m = 0.0f;
 #pragma unroll
         for (int c = 0; c < NR; ++c) {
-            acc[r][c] = __fdiv_rn(acc[r][c], sc[c]);
-            m = fmaxf(m, fabsf(acc[r][c]));
+            ACC(r, c) = __fmul_rn(ACC(r, c), rs[c]);
+            m = fmaxf(m, fabsf(ACC(r, c)));
         }
         m = group_max<16>(m);
         const float sigma = __fdiv_rn(m, 127.0f);
+        const float rho = (m > 0.0f) ? __fdiv_rn(127.0f, m) : 0.0f;
         if (tx == 0) w.row_scale[(size_t)u * D + row_of(r)] = sigma;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             uint32_t word = 0;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float code = 0.0f;
-                if (sigma > 0.0f) code = fminf(fmaxf(rintf(__fdiv_rn(acc[r][g * 4 + c], sigma)), -127.0f), 127.0f);
+                const float code = fminf(fmaxf(rintf(__fmul_rn(ACC(r, g * 4 + c), rho)), -127.0f), 127.0f);
                 word |= (uint32_t)((int)code & 0xff) << (8 * c);
             }
             *reinterpret_cast<uint32_t *>(Qu + (size_t)row_of(r) * D + g * 64 + tx * 4) = word;
@@ -324,6 +335,7 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
         const int gd = KDA ? D : 1;
         for (int j = tid; j < gd; j += kEncThreads) w.gate_sum[(size_t)u * gd + j] = 0.0;
     }
+#undef ACC
 }
 
 template <int D, bool KDA, typename KeyT>

@@ -1,0 +1,50 @@
+"""Run a short, fixed sequence of liblq launches for a profiler to capture.
+
+    python -m recurrent_state_quantization_lq_b200.profile_case [--workload NAME]
+        [--mode window|fp32|naive] [--tokens T] [--flush]
+
+Sets up one layer-state of the workload (prefill from a seeded FP32 state),
+then runs T decode launches (the windowed kernel sees 0..T-1 buffered tokens)
+and, with --flush, one window flush.  Launch order: the prefill's encode
+launch (windowed/naive modes), then the T decode launches, then the flush.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from recurrent_state_quantization_lq_b200 import inputs, lq
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="gdn_b64_h32_d128_w64", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--mode", default="window", choices=["window", "fp32", "naive"])
+    ap.add_argument("--tokens", type=int, default=34)
+    ap.add_argument("--flush", action="store_true")
+    args = ap.parse_args()
+    wl = inputs.WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T = min(args.tokens, wl.window) if args.mode == "window" else args.tokens
+    tb = inputs.tokens_on_device(wl.seed, T, wl.batch, wl.heads, wl.d_k, wl.d_v, wl.per_channel_gate, wl.dtype, dev)
+    S0 = 0.3 * torch.randn(wl.batch, wl.heads, wl.d_v, wl.d_k, device=dev,
+                           generator=torch.Generator(device=dev).manual_seed(wl.seed))
+    st = lq.DecodeState(wl.batch, wl.heads, wl.d_k, window=wl.window, n_comp_rows=wl.n_comp_rows,
+                        n_comp_cols=wl.n_comp_cols, gate="channel" if wl.per_channel_gate else "scalar",
+                        mode=args.mode, in_dtype=wl.dtype, device=dev)
+    st.prefill(S0)
+    out = torch.empty(wl.batch, wl.heads, wl.d_v, dtype=torch.float32, device=dev)
+    for t in range(T):
+        st.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=out)
+    if args.flush:
+        st.flush()
+    status = st.device_status()
+    if status != lq.LQ_OK:
+        raise lq.LQError(status, "profile_case")
+    print(f"profile_case: {wl.name} mode={args.mode} tokens={T} flush={args.flush} ok")
+
+
+if __name__ == "__main__":
+    main()

@@ -73,3 +73,62 @@ def compare_codes(q_gpu: np.ndarray, q_ref: np.ndarray) -> tuple[float, int]:
     """(fraction of equal codes, largest code difference)."""
     d = np.abs(q_gpu.astype(np.int32) - q_ref.astype(np.int32))
     return float((d == 0).mean()), int(d.max()) if d.size else 0
+
+
+def import_encoded(st: lq.DecodeState, ref: oracle.RunResult, f: int, units=None) -> None:
+    """Write the oracle's f-th encoded state into the GPU workspace (all units,
+    or the listed flattened units).  The window buffer must be empty."""
+    B, H, d = st.batch, st.heads, st.d
+    units = list(range(B * H)) if units is None else list(units)
+    sel = torch.tensor(units, dtype=torch.long)
+    dev = st.device
+
+    def put(name, arr):
+        v = st.view(name)
+        flat = v.view(B * H, *v.shape[2:])
+        flat[sel.to(dev)] = torch.as_tensor(np.ascontiguousarray(arr)).to(dev, flat.dtype).reshape(
+            len(units), *flat.shape[1:])
+
+    put("codes", ref.Q[:, f])
+    put("row_scale", ref.sigma[:, f])
+    if st.view("col_smooth") is not None:
+        put("col_smooth", ref.s[:, f])
+    nr, nc = st.cfg.n_comp_rows, st.cfg.n_comp_cols
+    if st.cfg.mode == 0 and nr + nc > 0:
+        idx = np.zeros((len(units), st.layout.comp_index_stride), np.int32)
+        idx[:, :nr + nc] = ref.idx[:, f]
+        put("comp_index", idx)
+        if nr:
+            put("comp_row_vec", ref.vec[:, f, :nr * d].reshape(len(units), nr, d))
+        if nc:
+            put("comp_col_vec", ref.vec[:, f, nr * d:].reshape(len(units), nc, d))
+    torch.cuda.synchronize()
+
+
+def decoded_state(ref: oracle.RunResult, f: int, nr: int, nc: int, d: int) -> np.ndarray:
+    """S~ = sigma Q s + C of the oracle's f-th encoding, [n, d, d] FP64."""
+    S = ref.sigma[:, f].astype(np.float64)[:, :, None] * ref.Q[:, f] * ref.s[:, f].astype(np.float64)[:, None, :]
+    for n in range(S.shape[0]):
+        for c in range(nr):
+            S[n, ref.idx[n, f, c], :] += ref.vec[n, f, c * d:(c + 1) * d]
+        for c in range(nc):
+            S[n, :, ref.idx[n, f, nr + c]] += ref.vec[n, f, nr * d + c * d:nr * d + (c + 1) * d]
+    return S
+
+
+def selection_is_near_tie(S_pre: np.ndarray, got_idx, ref_idx, nr: int, select: str = "l2",
+                          rtol: float = 1e-5) -> bool:
+    """Both compensator selections rank equally well on the oracle's FP32
+    pre-flush state up to rtol (a legitimate alternative at a near-tie)."""
+    R = S_pre.astype(np.float32).astype(np.float64)
+    def score(M, axis):
+        return (M ** 2).sum(axis=axis) if select == "l2" else np.abs(M).max(axis=axis)
+    rows = score(R, 1)
+    g_rows, r_rows = list(got_idx[:nr]), list(ref_idx[:nr])
+    if not np.allclose(np.sort(rows[g_rows]), np.sort(rows[r_rows]), rtol=rtol, atol=0):
+        return False
+    Rz = R.copy()
+    Rz[r_rows, :] = 0.0
+    cols = score(Rz, 0)
+    g_cols, r_cols = list(got_idx[nr:]), list(ref_idx[nr:])
+    return bool(np.allclose(np.sort(cols[g_cols]), np.sort(cols[r_cols]), rtol=rtol, atol=0))

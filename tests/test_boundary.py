@@ -54,7 +54,7 @@ def test_layout_regions_disjoint_aligned(mode, gate, d):
 
 
 @pytest.mark.parametrize("field,value", [("d_k", 96), ("d_v", 64), ("window", 0), ("window", 5000),
-                                         ("n_comp_rows", 17), ("n_comp_cols", -1), ("gate", 2),
+                                         ("n_comp_rows", 9), ("n_comp_cols", -1), ("gate", 2),
                                          ("mode", 3), ("smooth", 2), ("select", 2), ("in_dtype", 3),
                                          ("batch", 0), ("heads", 0)])
 def test_invalid_configs_rejected(field, value):

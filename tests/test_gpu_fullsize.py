@@ -12,7 +12,7 @@ import torch
 import oracle
 from recurrent_state_quantization_lq_b200 import inputs, lq
 
-from harness import compare_codes, gpu_run, oracle_params, rel_l2, to_device, unit_inputs
+from harness import compare_codes, gpu_run, import_encoded, oracle_params, rel_l2, to_device, unit_inputs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -34,7 +34,8 @@ def _run(wl: inputs.Workload, decode_tokens: int, n_sample: int):
                         gate=gate, in_dtype=wl.dtype, device=DEV)
     st.prefill(S0)
     first_codes = st.view("codes").cpu().clone()
-    o_gpu, shots = gpu_run(st, to_device(tb_dec, DEV), flush_every=W)
+    tbd = to_device(tb_dec, DEV)
+    o_gpu, shots = gpu_run(st, tbd, flush_every=W)
     assert st.device_status() == lq.LQ_OK
 
     # properties of the whole output and state
@@ -58,10 +59,24 @@ def _run(wl: inputs.Workload, decode_tokens: int, n_sample: int):
     o_s = o_gpu.reshape(decode_tokens, B * H, d)[:, units].transpose(0, 1).numpy()
     err = rel_l2(o_s, ref.o)
     assert err <= 1e-3, err
-    codes = [first_codes] + [s["codes"] for s in shots]
-    for f, c in enumerate(codes):
+    # codes of the prefill encoding and of the first flush (no cascade before it)
+    for f, c in enumerate([first_codes, shots[0]["codes"]]):
         frac, worst = compare_codes(c.reshape(B * H, d, d)[units].numpy(), ref.Q[:, f])
         assert frac >= 0.999 and worst <= 1, (f, frac, worst)
+
+    # teacher-forced window: the sampled units restart from the oracle's encoding
+    st.prefill(S0)
+    import_encoded(st, ref, 0, units)
+    o_w, snaps = gpu_run(st, inputs.TokenBatch(*(x[:W] for x in (tbd.q, tbd.k, tbd.v, tbd.g, tbd.beta))),
+                         flush_every=W)
+    o_ws = o_w.reshape(W, B * H, d)[:, units].transpose(0, 1).numpy()
+    assert rel_l2(o_ws, ref.o[:, :W]) <= 1e-5
+    c = snaps[0]["codes"].reshape(B * H, d, d)[units].numpy()
+    idx = snaps[0]["comp_index"].reshape(B * H, -1)[units].numpy()[:, :wl.n_comp_rows + wl.n_comp_cols]
+    keep = (idx == ref.idx[:, 1]).all(axis=1)
+    assert keep.sum() >= len(units) - 1
+    frac, worst = compare_codes(c[keep], ref.Q[keep, 1])
+    assert frac >= 0.999 and worst <= 1, (frac, worst)
     return err
 
 

@@ -17,7 +17,8 @@ import torch
 import oracle
 from recurrent_state_quantization_lq_b200 import inputs, lq
 
-from harness import compare_codes, gpu_run, oracle_params, rel_l2, snapshot, to_device, unit_inputs
+from harness import (compare_codes, decoded_state, gpu_run, import_encoded, oracle_params, rel_l2,
+                     selection_is_near_tie, snapshot, to_device, unit_inputs)
 
 pytestmark = pytest.mark.gpu
 
@@ -60,6 +61,9 @@ def test_prefill_codec_bit_exact(d, kind, comps, smooth, select):
         np.testing.assert_array_equal(got["codes"][b, h].numpy(), e.Q)
         np.testing.assert_array_equal(got["row_scale"][b, h].numpy(), e.sigma)
         np.testing.assert_array_equal(got["col_smooth"][b, h].numpy(), e.s)
+        if nr + nc == 0:
+            assert got["comp_index"] is None
+            continue
         idx = got["comp_index"][b, h].numpy()
         np.testing.assert_array_equal(idx[:nr], e.comp_rows)
         np.testing.assert_array_equal(idx[nr:nr + nc], e.comp_cols)
@@ -86,34 +90,60 @@ def test_naive_prefill_bit_exact(d):
 # ------------------------------------------------------------ windowed decode
 
 def _window_case(d, gate, dtype, W, nr, nc, B, H, T, seed, S0_kind="zero", smooth=1, select="l2"):
+    """Free-running: GPU and oracle each run their own trajectory from the same S0.
+    Teacher-forced: every GPU window starts from the oracle's encoded state."""
     tb = inputs.tokens(seed, 0, T, B, H, d, d, per_channel_gate=(gate == "channel"), dtype=dtype)
+    tbd = to_device(tb, DEV)
     S0 = _state(S0_kind, seed, B, H, d)
     st = lq.DecodeState(B, H, d, window=W, n_comp_rows=nr, n_comp_cols=nc, gate=gate, in_dtype=dtype,
                         smooth=smooth, select=select, device=DEV)
     st.prefill(S0.to(DEV).contiguous())
-    o_gpu, shots = gpu_run(st, to_device(tb, DEV), flush_every=W)
+    o_free, shots = gpu_run(st, tbd, flush_every=W)
     assert st.device_status() == lq.LQ_OK
     p = oracle_params(d, W, nr, nc, gate, "window", smooth, select)
-    units = range(B * H)
-    q, k, v, g, beta = unit_inputs(tb, units)
+    q, k, v, g, beta = unit_inputs(tb, range(B * H))
     ref = oracle.run(p, S0.reshape(B * H, d, d).double().numpy(), q, k, v, g, beta)
-    return o_gpu, shots, ref
 
-
-def _check_window(o_gpu, shots, ref, B, H, d, out_tol=1e-3):
-    T = o_gpu.shape[0]
+    # free-running: outputs over the whole run, codes at the first flush
     o_ref = ref.o.reshape(B, H, T, d).transpose(2, 0, 1, 3)
-    err = rel_l2(o_gpu.numpy(), o_ref)
-    assert err <= out_tol, err
-    for f, snap in enumerate(shots):
-        q_gpu = snap["codes"].reshape(B * H, d, d).numpy()
-        q_ref = ref.Q[:, f + 1]
-        frac, worst = compare_codes(q_gpu, q_ref)
-        assert frac >= 0.999 and worst <= 1, (f, frac, worst)
-        same = q_gpu == q_ref
-        sig_g = snap["row_scale"].reshape(B * H, d).numpy()
-        rows_same = same.all(axis=2)
-        np.testing.assert_allclose(sig_g[rows_same], ref.sigma[:, f + 1][rows_same], rtol=1e-4)
+    err = rel_l2(o_free.numpy(), o_ref)
+    assert err <= 1e-3, err
+    if shots:
+        frac, worst = compare_codes(shots[0]["codes"].reshape(B * H, d, d).numpy(), ref.Q[:, 1])
+        assert frac >= 0.999 and worst <= 1, ("free-running first flush", frac, worst)
+
+    # teacher-forced: window by window from the oracle's state
+    plain = oracle_params(d, gate=gate, mode="fp32")
+    st.prefill(None)
+    for w in range(T // W):
+        import_encoded(st, ref, w)
+        sl = slice(w * W, (w + 1) * W)
+        o_w, snaps = gpu_run(st, inputs.TokenBatch(*(x[sl] for x in (tbd.q, tbd.k, tbd.v, tbd.g, tbd.beta))),
+                             flush_every=W)
+        assert st.device_status() == lq.LQ_OK
+        e_w = rel_l2(o_w.numpy(), o_ref[sl])
+        assert e_w <= 1e-5, ("teacher-forced outputs", w, e_w)
+        snap = snaps[0]
+        got_idx = snap["comp_index"].reshape(B * H, -1).numpy()[:, :nr + nc] if nr + nc else None
+        codes = snap["codes"].reshape(B * H, d, d).numpy()
+        keep = np.ones(B * H, bool)
+        if nr + nc:
+            flips = np.nonzero((got_idx != ref.idx[:, w + 1]).any(axis=1))[0]
+            if len(flips):
+                S_tilde = decoded_state(ref, w, nr, nc, d)
+                pre = oracle.run(plain, S_tilde[flips], q[flips, sl], k[flips, sl], v[flips, sl], g[flips, sl],
+                                 beta[flips, sl], snapshots=False).S_final
+                for i, n in enumerate(flips):
+                    assert selection_is_near_tie(pre[i], got_idx[n], ref.idx[n, w + 1], nr, select), (w, n)
+                keep[flips] = False
+        frac, worst = compare_codes(codes[keep], ref.Q[keep, w + 1])
+        assert frac >= 0.999 and worst <= 1, ("teacher-forced flush", w, frac, worst)
+        same_rows = (codes == ref.Q[:, w + 1]).all(axis=2) & keep[:, None]
+        sig = snap["row_scale"].reshape(B * H, d).numpy()
+        np.testing.assert_allclose(sig[same_rows], ref.sigma[:, w + 1][same_rows], rtol=1e-5)
+        if nr + nc:
+            np.testing.assert_allclose(snap["col_smooth"].reshape(B * H, d).numpy()[keep],
+                                       ref.s[keep, w + 1], rtol=1e-5)
     return err
 
 
@@ -121,10 +151,8 @@ def _check_window(o_gpu, shots, ref, B, H, d, out_tol=1e-3):
 def test_tiny_gdn_workload(dtype):
     """One sequence, one 64x64 head from a zero state, 256 tokens, W = 64, 2+2 compensators."""
     wl = inputs.WORKLOADS["gdn_tiny_d64"]
-    o_gpu, shots, ref = _window_case(64, "scalar", dtype, wl.window, wl.n_comp_rows, wl.n_comp_cols,
-                                     wl.batch, wl.heads, wl.decode_tokens, wl.seed)
-    assert len(shots) == 4
-    _check_window(o_gpu, shots, ref, 1, 1, 64)
+    _window_case(64, "scalar", dtype, wl.window, wl.n_comp_rows, wl.n_comp_cols, wl.batch, wl.heads,
+                 wl.decode_tokens, wl.seed)
 
 
 @pytest.mark.parametrize("d", [64, 128])
@@ -133,17 +161,14 @@ def test_tiny_gdn_workload(dtype):
 def test_window_decode_variants(d, gate, W, nr, nc):
     B, H = 2, 3
     T = 2 * W + W // 2 + 1 if W > 1 else 9
-    o_gpu, shots, ref = _window_case(d, gate, torch.bfloat16, W, nr, nc, B, H, T, seed=11 + W,
-                                     S0_kind="normal")
-    _check_window(o_gpu, shots, ref, B, H, d)
+    _window_case(d, gate, torch.bfloat16, W, nr, nc, B, H, T, seed=11 + W, S0_kind="normal")
 
 
 def test_window_decode_planted_outliers_maxabs_nosmooth():
     d, B, H, W = 128, 2, 4, 16
     for smooth, select in ((0, "l2"), (1, "maxabs")):
-        o_gpu, shots, ref = _window_case(d, "scalar", torch.bfloat16, W, 2, 2, B, H, 3 * W, seed=5,
-                                         S0_kind="planted", smooth=smooth, select=select)
-        _check_window(o_gpu, shots, ref, B, H, d)
+        _window_case(d, "scalar", torch.bfloat16, W, 2, 2, B, H, 3 * W, seed=5, S0_kind="planted",
+                     smooth=smooth, select=select)
 
 
 def test_partial_window_flush_and_window_full():
@@ -212,5 +237,11 @@ def test_naive_int8_decode(d, gate):
                      *unit_inputs(tb, range(B * H)))
     o_ref = ref.o.reshape(B, H, T, d).transpose(2, 0, 1, 3)
     assert rel_l2(o_gpu.numpy(), o_ref) <= 1e-3
-    frac, worst = compare_codes(st.view("codes").reshape(-1, d, d).cpu().numpy(), ref.Q[:, -1])
-    assert frac >= 0.999 and worst <= 1, (frac, worst)
+    # teacher-forced: every token starts from the oracle's requantized state
+    tbd = to_device(tb, DEV)
+    for t in range(T):
+        import_encoded(st, ref, t)
+        o_t = st.decode_step(tbd.q[t], tbd.k[t], tbd.v[t], tbd.g[t], tbd.beta[t])
+        assert rel_l2(o_t.cpu().numpy(), o_ref[t]) <= 1e-5, t
+        frac, worst = compare_codes(st.view("codes").reshape(-1, d, d).cpu().numpy(), ref.Q[:, t + 1])
+        assert frac >= 0.999 and worst <= 1, (t, frac, worst)
