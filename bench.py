@@ -60,9 +60,9 @@ def decode_window_bytes(d: int, in_b: int, kda: bool, ncr: int, ncc: int, n_buf:
         fixed += 4 * d                       # kappa_t appended
         per_entry = 4 * d + 4 * d            # delta_j, kappa_j
     else:
-        fixed += 4 + 8 + 8 + 8               # g read, G read + written, G_t appended
+        fixed += 4 + 8 + 8 + 4               # g read, G read + written, exp(-G_t) appended
         fixed += in_b * d                    # k_t appended
-        per_entry = 4 * d + in_b * d + 8     # delta_j, k_j, G_j
+        per_entry = 4 * d + in_b * d + 4     # delta_j, k_j, exp(-G_j)
     return fixed + per_entry * n_buf
 
 
@@ -72,7 +72,7 @@ def flush_bytes(d: int, in_b: int, kda: bool, ncr: int, ncc: int, n_buf: int) ->
     cis = ((ncr + ncc + 3) // 4) * 4
     state = d * d + 8 * d + 4 * cis + 4 * d * (ncr + ncc)
     gd = d if kda else 1
-    entry = 4 * d + (4 * d if kda else in_b * d + 8)
+    entry = 4 * d + (4 * d if kda else in_b * d + 4)
     return 2 * state + 2 * 8 * gd + entry * n_buf
 
 

@@ -119,10 +119,10 @@ typedef struct lq_layout {
     size_t buf_delta;     /* f32   [N][window][d_v]  buffered delta_j             */
     size_t buf_key;       /* GDN: in_dtype [N][window][d_k] k_j;
                              KDA: f32 [N][window][d_k] k_j * exp(-G_j)            */
-    size_t buf_gate;      /* f64   [N][window_pad] G_j (GDN only)                 */
+    size_t buf_gate;      /* f32   [N][window_pad] exp(-G_j) (GDN only)           */
     size_t state_f32;     /* f32   [N][d_v][d_k]                  FP32 mode        */
     int32_t comp_index_stride;  /* n_comp_rows + n_comp_cols rounded up to 4      */
-    int32_t window_pad;         /* window rounded up to 2                          */
+    int32_t window_pad;         /* window rounded up to 4                          */
 } lq_layout;
 
 typedef struct lq_state_s *lq_handle;

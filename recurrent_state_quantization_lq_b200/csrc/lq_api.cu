@@ -71,7 +71,7 @@ void compute_layout(const lq_config *c, lq_layout *L) {
     } else {
         const int ncomp = c->n_comp_rows + c->n_comp_cols;
         L->comp_index_stride = ((ncomp + 3) / 4) * 4;
-        L->window_pad = ((c->window + 1) / 2) * 2;
+        L->window_pad = ((c->window + 3) / 4) * 4;
         const size_t gd = (c->gate == LQ_GATE_CHANNEL) ? d : 1;
         const size_t key_b = (c->gate == LQ_GATE_CHANNEL || c->in_dtype == LQ_DTYPE_F32) ? 4 : 2;
         L->codes = take(N * d * d);
@@ -83,7 +83,7 @@ void compute_layout(const lq_config *c, lq_layout *L) {
         L->gate_sum = take(N * gd * 8);
         L->buf_delta = take(N * (size_t)c->window * d * 4);
         L->buf_key = take(N * (size_t)c->window * d * key_b);
-        if (c->gate == LQ_GATE_SCALAR) L->buf_gate = take(N * (size_t)L->window_pad * 8);
+        if (c->gate == LQ_GATE_SCALAR) L->buf_gate = take(N * (size_t)L->window_pad * 4);
     }
     L->total_bytes = align256(off);
 }
@@ -126,7 +126,7 @@ lq::Views views(lq_handle h) {
     v.gate_sum = region<double>(b, L.gate_sum);
     v.buf_delta = region<float>(b, L.buf_delta);
     v.buf_key = region<void>(b, L.buf_key);
-    v.buf_gate = region<double>(b, L.buf_gate);
+    v.buf_gate = region<float>(b, L.buf_gate);
     v.state_f32 = region<float>(b, L.state_f32);
     v.comp_index_stride = L.comp_index_stride;
     v.window = h->cfg.window;

@@ -24,7 +24,7 @@ struct Views {
     double *gate_sum;
     float *buf_delta;
     void *buf_key;
-    double *buf_gate;
+    float *buf_gate;
     float *state_f32;
     int comp_index_stride;
     int window;
@@ -68,6 +68,16 @@ __device__ __forceinline__ float group_max(float x) {
 #pragma unroll
     for (int o = WIDTH / 2; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
     return x;
+}
+
+// exp(x) for a double x with |x| <= 80, to about two float ulps: expf of the
+// float-rounded argument, corrected to first order by the rounding remainder
+// (exp(xf + r) = exp(xf)(1 + r + O(r^2)) with |r| <= 2^-24 |x|).
+__device__ __forceinline__ float exp_of_double(double x) {
+    const float xf = (float)x;
+    const float r = (float)(x - (double)xf);
+    const float e = expf(xf);
+    return fmaf(e, r, e);
 }
 
 // ------------------------------------------------------------- error reporting

@@ -138,9 +138,9 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
             const int ne = min(kEncChunk, total - e0);
             if (!KDA && tid < ne) {
                 const int e = e0 + tid;
-                sh_fac[tid] = (e < ncomp)
-                                  ? (float)exp(GW_scalar)
-                                  : (float)exp(GW_scalar - w.buf_gate[(size_t)u * w.window_pad + (e - ncomp)]);
+                // buffered tokens carry omega_j = exp(-G_j): factor exp(G_W - G_j) = gamma_W omega_j
+                const float gW = (float)exp(GW_scalar);
+                sh_fac[tid] = (e < ncomp) ? gW : gW * w.buf_gate[(size_t)u * w.window_pad + (e - ncomp)];
             }
             __syncthreads();
             for (int idx = tid; idx < ne * D; idx += kEncThreads) {

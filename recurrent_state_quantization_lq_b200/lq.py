@@ -211,7 +211,7 @@ class DecodeState:
             "gate_sum": (torch.float64, (c.batch, c.heads, gd)),
             "buf_delta": (torch.float32, (c.batch, c.heads, c.window, d)),
             "buf_key": (key_dt, (c.batch, c.heads, c.window, d)),
-            "buf_gate": (torch.float64, (c.batch, c.heads, L.window_pad)),
+            "buf_gate": (torch.float32, (c.batch, c.heads, L.window_pad)),
             "state_f32": (torch.float32, (c.batch, c.heads, d, d)),
         }[name]
         dt, shape = spec

@@ -31,7 +31,7 @@ def test_layout_regions_disjoint_aligned(mode, gate, d):
              "comp_index": N * L.comp_index_stride * 4, "comp_row_vec": N * 3 * d * 4,
              "comp_col_vec": N * 1 * d * 4, "gate_sum": N * (d if gate == "channel" else 1) * 8,
              "buf_delta": N * 37 * d * 4, "buf_key": N * 37 * d * key_b,
-             "buf_gate": N * L.window_pad * 8, "state_f32": N * d * d * 4}
+             "buf_gate": N * L.window_pad * 4, "state_f32": N * d * d * 4}
     present = {
         "window": {"err", "codes", "row_scale", "col_smooth", "comp_index", "comp_row_vec", "comp_col_vec",
                    "gate_sum", "buf_delta", "buf_key"} | ({"buf_gate"} if gate == "scalar" else set()),
@@ -50,7 +50,7 @@ def test_layout_regions_disjoint_aligned(mode, gate, d):
     for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
         assert a1 <= b0
     if mode == "window":
-        assert L.comp_index_stride == 4 and L.window_pad == 38
+        assert L.comp_index_stride == 4 and L.window_pad == 40
 
 
 @pytest.mark.parametrize("field,value", [("d_k", 96), ("d_v", 64), ("window", 0), ("window", 5000),
