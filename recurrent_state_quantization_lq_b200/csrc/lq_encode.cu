@@ -1,17 +1,16 @@
-// State codec kernel: prefill ingestion and window flush.
+// State codec kernels: prefill ingestion and window flush.
 //
 // LeapQuant ("LeapQuant: Efficient Linear Attention with Accurate Recurrent
 // State Quantization", section "Abstract (arXiv)") quantizes the state only
 // once, at the end of each window; before that it keeps the state's largest
 // outliers as high-precision Compensator Tokens and smooths the remaining
-// residual.  One CTA per (sequence, head):
-//   1. rebuild the end-of-window state in FP32 registers,
-//        R = (R^ + C) diag(gamma_W) + sum_j delta_j (kappa_j * gamma_W)^T,
-//      a rank-(n_c + n_buf) update of the dequantized window-start state
-//      (compensators enter as buffered pairs with G = 0), or take the
-//      prefilled state as given;
-//   2. compensator rows (largest L2 norm, or max-abs), then columns of the
-//      row-zeroed residual, stored as FP32 pairs and zeroed;
+// residual.  Per (sequence, head) unit the codec
+//   1. takes the end-of-window state in FP32 registers: the prefilled state
+//      as given, or (flush) the rebuild
+//        R = (R^ + C + sum_j delta_j kappa_j^T) diag(gamma_W),
+//      a rank-n_buf update of the dequantized window-start state;
+//   2. takes compensator rows (largest L2 norm, or max-abs), then columns of
+//      the row-zeroed residual, stores them as FP32 pairs and zeroes them;
 //   3. s_j = sqrt(max_i |R_ij|) (1 for an empty column);
 //   4. R'_ij = R_ij * (1/s_j), M_i = max_j |R'_ij|, sigma_i = M_i / 127,
 //      Q_ij = rint(R'_ij * (127 / M_i)).
@@ -19,22 +18,50 @@
 // operations (square root, one division per column and per row, products
 // without fused adds), so a given FP32 state always encodes to the same codes,
 // scales and smoothing factors.
+//
+// The tile lives in registers: 256 threads in a 16 x 16 grid, thread (ty, tx)
+// owning rows g*64 + ty*4 + r and columns g*64 + tx*4 + c (g < d/64, r, c < 4),
+// as column pairs so the rank update runs on packed FP32 FMAs.
+//
+// The flush kernel is persistent and warp-specialized like the decode kernel:
+// a producer thread streams each unit's meta segment (scales, gate sums,
+// compensators), INT8 tile and buffered-entry chunks through a ring of 16 KB
+// shared-memory slots with 1-D bulk async copies and bounded mbarrier waits;
+// eight consumer warps rebuild, encode and store.
 #include "lq_kernels.h"
 
 namespace lq {
 namespace {
 
-constexpr int kEncThreads = 256;  // 16 x 16 thread grid over the d x d tile
-constexpr int kEncChunk = 16;     // buffered entries staged in shared memory per step
+constexpr int kTile = 256;                // threads holding the tile
+constexpr int kTileBarrier = 1;           // named barrier of those threads
+constexpr int kSlotBytes = 16384;
+constexpr int kSlots = 4;
+constexpr int kFlushThreads = kTile + 32; // + one producer warp
+constexpr int kMaxChunk = 16;
 
-template <int D>
-struct EncShape {
-    static constexpr int G = D / 64;   // 64-wide groups of rows / columns per thread
-    static constexpr int NR = 4 * G;   // rows (and columns) a thread owns
-    // thread (ty, tx) owns rows  g*64 + ty*4 + r  and columns  g*64 + tx*4 + c
-    static constexpr size_t smem_bytes =
-        sizeof(float) * (2 * kEncChunk * D + 16 * D + 3 * D + kEncChunk) + sizeof(int) * 32;
-};
+__host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+__device__ __forceinline__ void tile_sync() {
+    asm volatile("bar.sync %0, %1;" ::"r"(kTileBarrier), "r"(kTile) : "memory");
+}
+
+__device__ __forceinline__ bool tile_sync_or(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(kTileBarrier), "r"(kTile)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 // Warp-wide argmax over `n` scores with ties to the lower index; entries with
 // score < 0 are excluded.  Every lane returns the winner.
@@ -43,168 +70,65 @@ __device__ int warp_argmax(const float *score, int n) {
     float best = -1.0f;
     int bi = 0x7fffffff;
     for (int i = lane; i < n; i += 32) {
-        float s = score[i];
+        const float s = score[i];
         if (s > best) { best = s; bi = i; }   // i increases: strict '>' keeps the lower index
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-        float ob = __shfl_xor_sync(0xffffffffu, best, o);
-        int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
         if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
     }
     return bi;
 }
 
-template <int D, bool KDA, typename KeyT>
-__global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
-    using Sh = EncShape<D>;
-    constexpr int G = Sh::G, NR = Sh::NR;
-    const int u = blockIdx.x;
-    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-    const Views &w = a.w;
+// Codec scratch in shared memory (floats): per-ty column partials, scores,
+// reciprocal smoothing factors, selections.
+template <int D>
+struct CodecScratch {
+    static constexpr int PART = 0, SCORE = 16 * D, RS = 17 * D, SEL = 18 * D, FLOATS = 18 * D + 32;
+};
 
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    float *sh_delta = reinterpret_cast<float *>(smem_raw);    // [chunk][D]
-    float *sh_kap = sh_delta + kEncChunk * D;                   // [chunk][D]
-    float *sh_part = sh_kap + kEncChunk * D;                    // [16][D]
-    float *sh_gam = sh_part + 16 * D;                           // [D] gamma_W per key channel
-    float *sh_score = sh_gam + D;                               // [D]
-    float *sh_s = sh_score + D;                                 // [D] 1 / smoothing factor
-    float *sh_fac = sh_s + D;                                   // [chunk]
-    int *sh_sel = reinterpret_cast<int *>(sh_fac + kEncChunk);  // [32]: rows then columns
+template <int D>
+struct Tile {
+    static constexpr int G = D / 64;
+    static constexpr int NR = 4 * G;      // rows (and columns) a thread owns
+    float2 acc[NR][NR / 2];
+    int tx, ty, tid;
+    __device__ __forceinline__ int row(int r) const { return (r >> 2) * 64 + ty * 4 + (r & 3); }
+    __device__ __forceinline__ int col(int c) const { return (c >> 2) * 64 + tx * 4 + (c & 3); }
+    __device__ __forceinline__ float &at(int r, int c) { return (c & 1) ? acc[r][c >> 1].y : acc[r][c >> 1].x; }
+};
 
-    auto row_of = [&](int r) { return (r >> 2) * 64 + ty * 4 + (r & 3); };
-    auto col_of = [&](int c) { return (c >> 2) * 64 + tx * 4 + (c & 3); };
-
-    // The tile lives in registers as column pairs so the rank update can use
-    // packed FP32 FMAs; ACC(r, c) names one element.
-    float2 acc2[NR][NR / 2];
-#define ACC(r, c) ((((c) & 1) != 0) ? acc2[r][(c) >> 1].y : acc2[r][(c) >> 1].x)
-
-    // ------------------------------------------------------------ 1. rebuild
-    if (!a.from_buffer) {
-        if (a.S0 != nullptr) {
-            const float *S0 = a.S0 + (size_t)u * D * D;
-#pragma unroll
-            for (int r = 0; r < NR; ++r)
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    float4 x = *reinterpret_cast<const float4 *>(S0 + (size_t)row_of(r) * D + g * 64 + tx * 4);
-                    ACC(r, g * 4 + 0) = x.x; ACC(r, g * 4 + 1) = x.y;
-                    ACC(r, g * 4 + 2) = x.z; ACC(r, g * 4 + 3) = x.w;
-                }
-        } else {
-#pragma unroll
-            for (int r = 0; r < NR; ++r)
-#pragma unroll
-                for (int c = 0; c < NR; ++c) ACC(r, c) = 0.0f;
-        }
-    } else {
-        // gamma_W per key channel (scalar gate: one value for all)
-        double GW_scalar = 0.0;
-        if (KDA) {
-            for (int j = tid; j < D; j += kEncThreads) sh_gam[j] = (float)exp(w.gate_sum[(size_t)u * D + j]);
-        } else {
-            GW_scalar = w.gate_sum[u];
-            for (int j = tid; j < D; j += kEncThreads) sh_gam[j] = (float)exp(GW_scalar);
-        }
-        __syncthreads();
-        // dequantized window-start state, decayed: sigma_i Q_ij (s_j gamma_j)
-        const int8_t *Qu = w.codes + (size_t)u * D * D;
-        const float *sig = w.row_scale + (size_t)u * D;
-        const float *sm = w.col_smooth + (size_t)u * D;
-        float sg[NR];
-#pragma unroll
-        for (int c = 0; c < NR; ++c) sg[c] = sm[col_of(c)] * sh_gam[col_of(c)];
-#pragma unroll
-        for (int r = 0; r < NR; ++r) {
-            const float si = sig[row_of(r)];
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                uint32_t word = *reinterpret_cast<const uint32_t *>(Qu + (size_t)row_of(r) * D + g * 64 + tx * 4);
-                float f0, f1, f2, f3;
-                i8x4_to_f32(word, f0, f1, f2, f3);
-                ACC(r, g * 4 + 0) = (si * f0) * sg[g * 4 + 0];
-                ACC(r, g * 4 + 1) = (si * f1) * sg[g * 4 + 1];
-                ACC(r, g * 4 + 2) = (si * f2) * sg[g * 4 + 2];
-                ACC(r, g * 4 + 3) = (si * f3) * sg[g * 4 + 3];
-            }
-        }
-        // compensators (entries with G = 0), then the buffered tokens
-        const int ncomp = w.n_comp_rows + w.n_comp_cols;
-        const int total = ncomp + a.n_buf;
-        const int32_t *cidx = w.comp_index + (size_t)u * w.comp_index_stride;
-        for (int e0 = 0; e0 < total; e0 += kEncChunk) {
-            const int ne = min(kEncChunk, total - e0);
-            if (!KDA && tid < ne) {
-                const int e = e0 + tid;
-                // buffered tokens carry omega_j = exp(-G_j): factor exp(G_W - G_j) = gamma_W omega_j
-                const float gW = (float)exp(GW_scalar);
-                sh_fac[tid] = (e < ncomp) ? gW : gW * w.buf_gate[(size_t)u * w.window_pad + (e - ncomp)];
-            }
-            __syncthreads();
-            for (int idx = tid; idx < ne * D; idx += kEncThreads) {
-                const int el = idx / D, j = idx - el * D, e = e0 + el;
-                float dv, kv;
-                if (e < w.n_comp_rows) {                       // row compensator (e_i, k_c)
-                    dv = (j == cidx[e]) ? 1.0f : 0.0f;
-                    kv = w.comp_row_vec[((size_t)u * w.n_comp_rows + e) * D + j] * sh_gam[j];
-                } else if (e < ncomp) {                        // column compensator (v_c, e_j)
-                    const int c = e - w.n_comp_rows;
-                    dv = w.comp_col_vec[((size_t)u * w.n_comp_cols + c) * D + j];
-                    kv = (j == cidx[w.n_comp_rows + c]) ? sh_gam[j] : 0.0f;
-                } else {                                       // buffered token
-                    const size_t slot = (size_t)u * w.window + (e - ncomp);
-                    dv = w.buf_delta[slot * D + j];
-                    if (KDA) {
-                        kv = reinterpret_cast<const float *>(w.buf_key)[slot * D + j] * sh_gam[j];
-                    } else {
-                        const KeyT *kp = reinterpret_cast<const KeyT *>(w.buf_key) + slot * D + j;
-                        kv = static_cast<float>(*kp) * sh_fac[el];
-                    }
-                }
-                sh_delta[el * D + j] = dv;
-                sh_kap[el * D + j] = kv;
-            }
-            __syncthreads();
-            for (int el = 0; el < ne; ++el) {
-                float dr[NR];
-                float2 kc[NR / 2];
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    float4 x = *reinterpret_cast<const float4 *>(sh_delta + el * D + g * 64 + ty * 4);
-                    float4 y = *reinterpret_cast<const float4 *>(sh_kap + el * D + g * 64 + tx * 4);
-                    dr[g * 4 + 0] = x.x; dr[g * 4 + 1] = x.y; dr[g * 4 + 2] = x.z; dr[g * 4 + 3] = x.w;
-                    kc[g * 2 + 0] = make_float2(y.x, y.y);
-                    kc[g * 2 + 1] = make_float2(y.z, y.w);
-                }
-#pragma unroll
-                for (int r = 0; r < NR; ++r) {
-                    const float2 dd = make_float2(dr[r], dr[r]);
-#pragma unroll
-                    for (int m = 0; m < NR / 2; ++m) acc2[r][m] = __ffma2_rn(dd, kc[m], acc2[r][m]);
-                }
-            }
-            __syncthreads();
-        }
-    }
+// Steps 2-4 of the codec on the tile in registers, plus the stores.  Called by
+// exactly the kTile tile threads (tid < kTile).
+template <int D, bool KDA>
+__device__ void codec_store(Tile<D> &T, int u, const Views &w, int n_rows, int n_cols, int smooth, int select,
+                            float *scratch) {
+    using CS = CodecScratch<D>;
+    constexpr int G = Tile<D>::G, NR = Tile<D>::NR;
+    float *sh_part = scratch + CS::PART, *sh_score = scratch + CS::SCORE, *sh_rs = scratch + CS::RS;
+    int *sh_sel = reinterpret_cast<int *>(scratch + CS::SEL);
+    const int tid = T.tid, tx = T.tx, ty = T.ty;
+    const bool l2 = (select == LQ_SELECT_L2);
+    tile_sync();   // the scratch of the previous unit is free
 
     // ------------------------------------------------- 2a. compensator rows
-    if (a.n_rows > 0) {
+    if (n_rows > 0) {
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
             float p = 0.0f;
 #pragma unroll
             for (int c = 0; c < NR; ++c) {
-                const float x = fabsf(ACC(r, c));
-                p = (a.select == LQ_SELECT_L2) ? p + x * x : fmaxf(p, x);
+                const float x = fabsf(T.at(r, c));
+                p = l2 ? p + x * x : fmaxf(p, x);
             }
-            p = (a.select == LQ_SELECT_L2) ? group_sum<16>(p) : group_max<16>(p);
-            if (tx == 0) sh_score[row_of(r)] = p;
+            p = l2 ? group_sum<16>(p) : group_max<16>(p);
+            if (tx == 0) sh_score[T.row(r)] = p;
         }
-        __syncthreads();
+        tile_sync();
         if (tid < 32) {
-            for (int c = 0; c < a.n_rows; ++c) {
+            for (int c = 0; c < n_rows; ++c) {
                 const int i = warp_argmax(sh_score, D);
                 if (tid == 0) {
                     sh_sel[c] = i;
@@ -214,68 +138,68 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
                 __syncwarp();
             }
         }
-        __syncthreads();
+        tile_sync();
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
-            for (int c = 0; c < a.n_rows; ++c) {
-                if (sh_sel[c] == row_of(r)) {
-                    float *dst = w.comp_row_vec + ((size_t)u * a.n_rows + c) * D;
+            for (int c = 0; c < n_rows; ++c) {
+                if (sh_sel[c] == T.row(r)) {
+                    float *dst = w.comp_row_vec + ((size_t)u * n_rows + c) * D;
 #pragma unroll
                     for (int g = 0; g < G; ++g)
                         *reinterpret_cast<float4 *>(dst + g * 64 + tx * 4) =
-                            make_float4(ACC(r, g * 4), ACC(r, g * 4 + 1), ACC(r, g * 4 + 2), ACC(r, g * 4 + 3));
+                            make_float4(T.at(r, g * 4), T.at(r, g * 4 + 1), T.at(r, g * 4 + 2), T.at(r, g * 4 + 3));
 #pragma unroll
-                    for (int cc = 0; cc < NR; ++cc) ACC(r, cc) = 0.0f;
+                    for (int m = 0; m < NR / 2; ++m) T.acc[r][m] = make_float2(0.0f, 0.0f);
                 }
             }
         }
     }
 
     // ---------------------------------------------- 2b. compensator columns
-    if (a.n_cols > 0) {
+    if (n_cols > 0) {
 #pragma unroll
         for (int c = 0; c < NR; ++c) {
             float p = 0.0f;
 #pragma unroll
             for (int r = 0; r < NR; ++r) {
-                const float x = fabsf(ACC(r, c));
-                p = (a.select == LQ_SELECT_L2) ? p + x * x : fmaxf(p, x);
+                const float x = fabsf(T.at(r, c));
+                p = l2 ? p + x * x : fmaxf(p, x);
             }
-            sh_part[ty * D + col_of(c)] = p;
+            sh_part[ty * D + T.col(c)] = p;
         }
-        __syncthreads();
-        for (int j = tid; j < D; j += kEncThreads) {
+        tile_sync();
+        for (int j = tid; j < D; j += kTile) {
             float p = 0.0f;
             for (int y = 0; y < 16; ++y) {
                 const float x = sh_part[y * D + j];
-                p = (a.select == LQ_SELECT_L2) ? p + x : fmaxf(p, x);
+                p = l2 ? p + x : fmaxf(p, x);
             }
             sh_score[j] = p;
         }
-        __syncthreads();
+        tile_sync();
         if (tid < 32) {
-            for (int c = 0; c < a.n_cols; ++c) {
+            for (int c = 0; c < n_cols; ++c) {
                 const int j = warp_argmax(sh_score, D);
                 if (tid == 0) {
                     sh_sel[16 + c] = j;
                     sh_score[j] = -1.0f;
-                    w.comp_index[(size_t)u * w.comp_index_stride + a.n_rows + c] = j;
+                    w.comp_index[(size_t)u * w.comp_index_stride + n_rows + c] = j;
                 }
                 __syncwarp();
             }
         }
-        __syncthreads();
+        tile_sync();
 #pragma unroll
         for (int c = 0; c < NR; ++c) {
-            for (int cc = 0; cc < a.n_cols; ++cc) {
-                if (sh_sel[16 + cc] == col_of(c)) {
-                    float *dst = w.comp_col_vec + ((size_t)u * a.n_cols + cc) * D;
+            for (int cc = 0; cc < n_cols; ++cc) {
+                if (sh_sel[16 + cc] == T.col(c)) {
+                    float *dst = w.comp_col_vec + ((size_t)u * n_cols + cc) * D;
 #pragma unroll
                     for (int g = 0; g < G; ++g)
-                        *reinterpret_cast<float4 *>(dst + g * 64 + ty * 4) =
-                            make_float4(ACC(g * 4, c), ACC(g * 4 + 1, c), ACC(g * 4 + 2, c), ACC(g * 4 + 3, c));
+                        *reinterpret_cast<float4 *>(dst + g * 64 + ty * 4) = make_float4(
+                            T.at(g * 4, c), T.at(g * 4 + 1, c), T.at(g * 4 + 2, c), T.at(g * 4 + 3, c));
 #pragma unroll
-                    for (int r = 0; r < NR; ++r) ACC(r, c) = 0.0f;
+                    for (int r = 0; r < NR; ++r) T.at(r, c) = 0.0f;
                 }
             }
         }
@@ -286,62 +210,398 @@ __global__ void __launch_bounds__(kEncThreads, 2) encode_kernel(EncodeArgs a) {
     for (int c = 0; c < NR; ++c) {
         float m = 0.0f;
 #pragma unroll
-        for (int r = 0; r < NR; ++r) m = fmaxf(m, fabsf(ACC(r, c)));
-        sh_part[ty * D + col_of(c)] = m;
+        for (int r = 0; r < NR; ++r) m = fmaxf(m, fabsf(T.at(r, c)));
+        sh_part[ty * D + T.col(c)] = m;
     }
-    __syncthreads();
-    for (int j = tid; j < D; j += kEncThreads) {
+    tile_sync();
+    for (int j = tid; j < D; j += kTile) {
         float m = 0.0f;
         for (int y = 0; y < 16; ++y) m = fmaxf(m, sh_part[y * D + j]);
-        const float s = (a.smooth && m > 0.0f) ? __fsqrt_rn(m) : 1.0f;
-        sh_s[j] = __fdiv_rn(1.0f, s);          // applied as a multiplication
+        const float s = (smooth && m > 0.0f) ? __fsqrt_rn(m) : 1.0f;
+        sh_rs[j] = __fdiv_rn(1.0f, s);          // applied as a multiplication
         if (w.col_smooth != nullptr) w.col_smooth[(size_t)u * D + j] = s;
     }
-    __syncthreads();
+    tile_sync();
 
     // ------------------------------------------ 4. row scales and the codes
-    // R'_ij = R_ij * (1/s_j); M_i = max_j |R'_ij|; sigma_i = M_i / 127;
-    // Q_ij = rint(R'_ij * (127 / M_i)).
     float rs[NR];
 #pragma unroll
-    for (int c = 0; c < NR; ++c) rs[c] = sh_s[col_of(c)];
+    for (int c = 0; c < NR; ++c) rs[c] = sh_rs[T.col(c)];
     int8_t *Qu = w.codes + (size_t)u * D * D;
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
         float m = 0.0f;
 #pragma unroll
         for (int c = 0; c < NR; ++c) {
-            ACC(r, c) = __fmul_rn(ACC(r, c), rs[c]);
-            m = fmaxf(m, fabsf(ACC(r, c)));
+            T.at(r, c) = __fmul_rn(T.at(r, c), rs[c]);
+            m = fmaxf(m, fabsf(T.at(r, c)));
         }
         m = group_max<16>(m);
         const float sigma = __fdiv_rn(m, 127.0f);
         const float rho = (m > 0.0f) ? __fdiv_rn(127.0f, m) : 0.0f;
-        if (tx == 0) w.row_scale[(size_t)u * D + row_of(r)] = sigma;
+        if (tx == 0) w.row_scale[(size_t)u * D + T.row(r)] = sigma;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             uint32_t word = 0;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const float code = fminf(fmaxf(rintf(__fmul_rn(ACC(r, g * 4 + c), rho)), -127.0f), 127.0f);
+                const float code = fminf(fmaxf(rintf(__fmul_rn(T.at(r, g * 4 + c), rho)), -127.0f), 127.0f);
                 word |= (uint32_t)((int)code & 0xff) << (8 * c);
             }
-            *reinterpret_cast<uint32_t *>(Qu + (size_t)row_of(r) * D + g * 64 + tx * 4) = word;
+            *reinterpret_cast<uint32_t *>(Qu + (size_t)T.row(r) * D + g * 64 + tx * 4) = word;
         }
     }
 
     // -------------------------------------------- 5. start the next window
     if (w.gate_sum != nullptr) {
         const int gd = KDA ? D : 1;
-        for (int j = tid; j < gd; j += kEncThreads) w.gate_sum[(size_t)u * gd + j] = 0.0;
+        for (int j = tid; j < gd; j += kTile) w.gate_sum[(size_t)u * gd + j] = 0.0;
     }
-#undef ACC
+}
+
+// ================================================================== prefill
+
+template <int D, bool KDA>
+__global__ void __launch_bounds__(kTile, 2) prefill_kernel(EncodeArgs a) {
+    constexpr int G = Tile<D>::G, NR = Tile<D>::NR;
+    extern __shared__ __align__(16) float pf_scratch[];
+    Tile<D> T;
+    T.tid = threadIdx.x;
+    T.tx = T.tid & 15;
+    T.ty = T.tid >> 4;
+    const int u = blockIdx.x;
+    if (a.S0 != nullptr) {
+        const float *S0 = a.S0 + (size_t)u * D * D;
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float4 x = *reinterpret_cast<const float4 *>(S0 + (size_t)T.row(r) * D + g * 64 + T.tx * 4);
+                T.acc[r][g * 2] = make_float2(x.x, x.y);
+                T.acc[r][g * 2 + 1] = make_float2(x.z, x.w);
+            }
+    } else {
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+#pragma unroll
+            for (int m = 0; m < NR / 2; ++m) T.acc[r][m] = make_float2(0.0f, 0.0f);
+    }
+    codec_store<D, KDA>(T, u, a.w, a.n_rows, a.n_cols, a.smooth, a.select, pf_scratch);
+}
+
+// ==================================================================== flush
+
+template <int D, bool KDA, typename KeyT>
+struct FlushShape {
+    static constexpr int KB = (int)sizeof(KeyT);
+    static constexpr int ENTRY = 4 * D + KB * D + (KDA ? 0 : 4);
+    static constexpr int E0 = (kSlotBytes / ENTRY) & ~3;
+    static constexpr int E = E0 < kMaxChunk ? E0 : kMaxChunk;      // entries per chunk segment
+    static constexpr int C_KEY = 4 * D * E;                         // chunk: deltas, keys, omega_j
+    static constexpr int C_GATE = C_KEY + KB * D * E;
+    // shared memory: barriers, ring, staged keys (two buffers), codec scratch
+    static constexpr int OFF_RING = 128;
+    static constexpr int OFF_STAGE = OFF_RING + kSlots * kSlotBytes;
+    static constexpr int OFF_GAMMA = OFF_STAGE + (KDA ? 0 : 2 * kMaxChunk * D * 4);
+    static constexpr int OFF_CODEC = OFF_GAMMA + 4 * D;
+    static constexpr int SMEM = OFF_CODEC + 4 * CodecScratch<D>::FLOATS;
+    static_assert(E >= 4, "chunk size");
+};
+
+struct FlushMeta {
+    int sig, s, gsum, cidx, crow, ccol, bytes;
+};
+
+template <int D, bool KDA>
+__host__ __device__ FlushMeta flush_meta_layout(int ncr, int ncc, int cis) {
+    FlushMeta m{};
+    int o = 0;
+    m.sig = o;  o += 4 * D;
+    m.s = o;    o += 4 * D;
+    m.gsum = o; o += KDA ? 8 * D : 0;
+    m.cidx = o; o += (ncr + ncc) > 0 ? 4 * cis : 0;
+    m.crow = o; o += 4 * D * ncr;
+    m.ccol = o; o += 4 * D * ncc;
+    m.bytes = o;
+    return m;
+}
+
+template <int D, bool KDA, typename KeyT>
+__global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
+    using Sh = FlushShape<D, KDA, KeyT>;
+    constexpr int G = Tile<D>::G, NR = Tile<D>::NR, E = Sh::E;
+    const Views &w = a.w;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ncr = w.n_comp_rows, ncc = w.n_comp_cols, cis = w.comp_index_stride, ncomp = ncr + ncc;
+    const int n_buf = a.n_buf, nchunks = (n_buf + E - 1) / E, units = w.units;
+    const FlushMeta M = flush_meta_layout<D, KDA>(ncr, ncc, cis);
+
+    extern __shared__ __align__(128) unsigned char sm[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm);
+    uint64_t *empty = full + kSlots;
+    unsigned char *ring = sm + Sh::OFF_RING;
+    float *stage = reinterpret_cast<float *>(sm + Sh::OFF_STAGE);
+    float *sgam = reinterpret_cast<float *>(sm + Sh::OFF_GAMMA);     // gamma_W per key channel
+    float *scratch = reinterpret_cast<float *>(sm + Sh::OFF_CODEC);
+
+    if (tid == 0) {
+        for (int i = 0; i < kSlots; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kTile);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------------- producer
+    if (warp == kTile / 32) {
+        if (lane != 0) return;
+        const uint64_t stream_once = l2_policy_evict_first();
+        int slot = 0;
+        uint32_t ph = 0;
+        auto acquire = [&](int u, int detail) -> unsigned char * {
+            if (!mbar_wait(&empty[slot], ph ^ 1u, kWaitBudgetCycles)) {
+                report_error(w.err, LQ_DEVERR_TIMEOUT, u, detail);
+                return nullptr;
+            }
+            return ring + slot * kSlotBytes;
+        };
+        auto advance = [&]() {
+            if (++slot == kSlots) { slot = 0; ph ^= 1u; }
+        };
+        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+            unsigned char *dst = acquire(u, -1);
+            if (dst == nullptr) return;
+            uint64_t *bar = &full[slot];
+            mbar_arrive_expect_tx(bar, (uint32_t)M.bytes);
+            bulk_g2s(dst + M.sig, w.row_scale + (size_t)u * D, 4 * D, bar);
+            bulk_g2s(dst + M.s, w.col_smooth + (size_t)u * D, 4 * D, bar);
+            if (KDA) bulk_g2s(dst + M.gsum, w.gate_sum + (size_t)u * D, 8 * D, bar);
+            if (ncomp > 0) {
+                bulk_g2s(dst + M.cidx, w.comp_index + (size_t)u * cis, 4 * cis, bar);
+                if (ncr > 0) bulk_g2s(dst + M.crow, w.comp_row_vec + (size_t)u * ncr * D, 4 * D * ncr, bar);
+                if (ncc > 0) bulk_g2s(dst + M.ccol, w.comp_col_vec + (size_t)u * ncc * D, 4 * D * ncc, bar);
+            }
+            advance();
+            dst = acquire(u, -2);
+            if (dst == nullptr) return;
+            bar = &full[slot];
+            mbar_arrive_expect_tx(bar, D * D);
+            bulk_g2s_stream(dst, w.codes + (size_t)u * D * D, D * D, bar, stream_once);
+            advance();
+            for (int c = 0; c < nchunks; ++c) {
+                dst = acquire(u, -3 - c);
+                if (dst == nullptr) return;
+                const int e0 = c * E, ne = min(E, n_buf - e0);
+                const size_t first = (size_t)u * w.window + e0;
+                const uint32_t bd = 4u * ne * D, bk = (uint32_t)sizeof(KeyT) * ne * D;
+                const uint32_t bg = KDA ? 0u : 4u * (uint32_t)align_up(ne, 4);
+                bar = &full[slot];
+                mbar_arrive_expect_tx(bar, bd + bk + bg);
+                bulk_g2s_stream(dst, w.buf_delta + first * D, bd, bar, stream_once);
+                bulk_g2s_stream(dst + Sh::C_KEY, reinterpret_cast<const KeyT *>(w.buf_key) + first * D, bk, bar,
+                                stream_once);
+                if (!KDA) bulk_g2s(dst + Sh::C_GATE, w.buf_gate + (size_t)u * w.window_pad + e0, bg, bar);
+                advance();
+            }
+        }
+        return;
+    }
+
+    // ------------------------------------------------------------ tile threads
+    Tile<D> T;
+    T.tid = tid;
+    T.tx = tid & 15;
+    T.ty = tid >> 4;
+    int slot = 0;
+    uint32_t ph = 0;
+    auto advance = [&]() {
+        if (++slot == kSlots) { slot = 0; ph ^= 1u; }
+    };
+    int u = blockIdx.x;
+    double G_n = (!KDA && u < units) ? w.gate_sum[u] : 0.0;
+    for (; u < units; u += gridDim.x) {
+        const double GW = G_n;                       // scalar gate: G at the window end
+        if (!KDA && u + (int)gridDim.x < units) G_n = w.gate_sum[u + gridDim.x];
+
+        // -------- dequantized window-start state plus compensators (undecayed)
+        bool bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
+        const unsigned char *mp = ring + slot * kSlotBytes;
+        const int meta_slot = slot;
+        advance();
+        bad |= !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
+        const int8_t *sQ = reinterpret_cast<const int8_t *>(ring + slot * kSlotBytes);
+        const int q_slot = slot;
+        advance();
+        if (tile_sync_or(bad)) {
+            if (tid == 0) report_error(w.err, LQ_DEVERR_TIMEOUT, u, 0);
+            return;
+        }
+        {
+            const float *sig = reinterpret_cast<const float *>(mp + M.sig);
+            const float *sm_s = reinterpret_cast<const float *>(mp + M.s);
+            float sc[NR];
+#pragma unroll
+            for (int c = 0; c < NR; ++c) sc[c] = sm_s[T.col(c)];
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                const float si = sig[T.row(r)];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const uint32_t word = *reinterpret_cast<const uint32_t *>(sQ + T.row(r) * D + g * 64 + T.tx * 4);
+                    float f0, f1, f2, f3;
+                    i8x4_to_f32(word, f0, f1, f2, f3);
+                    T.acc[r][g * 2] = make_float2((si * f0) * sc[g * 4 + 0], (si * f1) * sc[g * 4 + 1]);
+                    T.acc[r][g * 2 + 1] = make_float2((si * f2) * sc[g * 4 + 2], (si * f3) * sc[g * 4 + 3]);
+                }
+            }
+            if (ncomp > 0) {
+                const int32_t *cidx = reinterpret_cast<const int32_t *>(mp + M.cidx);
+                const float *crow = reinterpret_cast<const float *>(mp + M.crow);
+                const float *ccol = reinterpret_cast<const float *>(mp + M.ccol);
+                for (int c = 0; c < ncr; ++c) {
+                    const int i = cidx[c];
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) {
+                        if (T.row(r) == i) {
+#pragma unroll
+                            for (int cc = 0; cc < NR; ++cc) T.at(r, cc) += crow[c * D + T.col(cc)];
+                        }
+                    }
+                }
+                for (int c = 0; c < ncc; ++c) {
+                    const int j = cidx[ncr + c];
+#pragma unroll
+                    for (int cc = 0; cc < NR; ++cc) {
+                        if (T.col(cc) == j) {
+#pragma unroll
+                            for (int r = 0; r < NR; ++r) T.at(r, cc) += ccol[c * D + T.row(r)];
+                        }
+                    }
+                }
+            }
+        }
+        // decay of the window: gamma_W per key channel (scalar gate: one value)
+        if (tid < D) {
+            sgam[tid] = KDA ? exp_of_double(reinterpret_cast<const double *>(mp + M.gsum)[tid]) : exp_of_double(GW);
+        }
+        mbar_arrive(&empty[meta_slot]);
+        mbar_arrive(&empty[q_slot]);
+
+        // -------- rank-n_buf update with the buffered entries
+        for (int c = 0; c < nchunks; ++c) {
+            bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
+            const unsigned char *cp = ring + slot * kSlotBytes;
+            const float *sDelta = reinterpret_cast<const float *>(cp);
+            const int ne = min(E, n_buf - c * E);
+            const float *kap;
+            if (KDA) {
+                kap = reinterpret_cast<const float *>(cp + Sh::C_KEY);
+            } else {
+                // stage omega_j k_j as FP32 (each key element converted once)
+                float *sb = stage + (c & 1) * kMaxChunk * D;
+                const KeyT *keys = reinterpret_cast<const KeyT *>(cp + Sh::C_KEY);
+                const float *omega = reinterpret_cast<const float *>(cp + Sh::C_GATE);
+                for (int idx = tid; idx < ne * (D / 8); idx += kTile) {
+                    const int el = idx / (D / 8), j0 = (idx % (D / 8)) * 8;
+                    const float om = omega[el];
+                    float kv[8];
+                    if constexpr (sizeof(KeyT) == 2) {
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(keys + el * D + j0);
+                        const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            kv[2 * h] = bf16_bits_to_f32(wd[h] & 0xffffu);
+                            kv[2 * h + 1] = bf16_bits_to_f32(wd[h] >> 16);
+                        }
+                    } else {
+                        const float4 x0 = *reinterpret_cast<const float4 *>(keys + el * D + j0);
+                        const float4 x1 = *reinterpret_cast<const float4 *>(keys + el * D + j0 + 4);
+                        kv[0] = x0.x; kv[1] = x0.y; kv[2] = x0.z; kv[3] = x0.w;
+                        kv[4] = x1.x; kv[5] = x1.y; kv[6] = x1.z; kv[7] = x1.w;
+                    }
+                    *reinterpret_cast<float4 *>(sb + el * D + j0) =
+                        make_float4(om * kv[0], om * kv[1], om * kv[2], om * kv[3]);
+                    *reinterpret_cast<float4 *>(sb + el * D + j0 + 4) =
+                        make_float4(om * kv[4], om * kv[5], om * kv[6], om * kv[7]);
+                }
+                kap = sb;
+            }
+            if (tile_sync_or(bad)) {
+                if (tid == 0) report_error(w.err, LQ_DEVERR_TIMEOUT, u, 1 + c);
+                return;
+            }
+            for (int el = 0; el < ne; ++el) {
+                float dr[NR];
+                float2 kc[NR / 2];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float4 x = *reinterpret_cast<const float4 *>(sDelta + el * D + g * 64 + T.ty * 4);
+                    const float4 y = *reinterpret_cast<const float4 *>(kap + el * D + g * 64 + T.tx * 4);
+                    dr[g * 4 + 0] = x.x; dr[g * 4 + 1] = x.y; dr[g * 4 + 2] = x.z; dr[g * 4 + 3] = x.w;
+                    kc[g * 2 + 0] = make_float2(y.x, y.y);
+                    kc[g * 2 + 1] = make_float2(y.z, y.w);
+                }
+#pragma unroll
+                for (int r = 0; r < NR; ++r) {
+                    const float2 dd = make_float2(dr[r], dr[r]);
+#pragma unroll
+                    for (int m = 0; m < NR / 2; ++m) T.acc[r][m] = __ffma2_rn(dd, kc[m], T.acc[r][m]);
+                }
+            }
+            mbar_arrive(&empty[slot]);
+            advance();
+        }
+
+        // -------- apply the window's decay
+        tile_sync();
+        {
+            float2 gg[NR / 2];
+#pragma unroll
+            for (int m = 0; m < NR / 2; ++m) gg[m] = make_float2(sgam[T.col(2 * m)], sgam[T.col(2 * m + 1)]);
+#pragma unroll
+            for (int r = 0; r < NR; ++r)
+#pragma unroll
+                for (int m = 0; m < NR / 2; ++m) T.acc[r][m] = __fmul2_rn(T.acc[r][m], gg[m]);
+        }
+        codec_store<D, KDA>(T, u, w, ncr, ncc, a.smooth, a.select, scratch);
+    }
+}
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
 }
 
 template <int D, bool KDA, typename KeyT>
 cudaError_t launch_encode_t(const EncodeArgs &a, cudaStream_t s) {
-    const size_t smem = EncShape<D>::smem_bytes;
-    encode_kernel<D, KDA, KeyT><<<a.w.units, kEncThreads, smem, s>>>(a);
+    if (!a.from_buffer) {
+        prefill_kernel<D, KDA><<<a.w.units, kTile, 4 * CodecScratch<D>::FLOATS, s>>>(a);
+        return cudaGetLastError();
+    }
+    using Sh = FlushShape<D, KDA, KeyT>;
+    const FlushMeta M = flush_meta_layout<D, KDA>(a.w.n_comp_rows, a.w.n_comp_cols, a.w.comp_index_stride);
+    if (M.bytes > kSlotBytes || D * D > kSlotBytes) return cudaErrorInvalidValue;
+    auto kern = flush_kernel<D, KDA, KeyT>;
+    static bool opted_in[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !opted_in[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::SMEM);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) opted_in[dev] = true;
+    }
+    const int grid = min(a.w.units, 2 * sm_count());
+    kern<<<grid, kFlushThreads, Sh::SMEM, s>>>(a);
     return cudaGetLastError();
 }
 
