@@ -1,5 +1,7 @@
 // liblq C ABI: config validation, workspace layout, handles and launches.
 // The declarations and the contract of every entry point are in include/lq.h.
+#include <cuda.h>
+
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -100,12 +102,14 @@ lq_status cuda_fail(cudaError_t e, const char *what) {
 }  // namespace
 
 struct lq_state_s {
+    CUtensorMap codes_map;   // INT8 tiles for the windowed decode (made at its first call)
     uint32_t magic;
     lq_config cfg;
     lq_layout lay;
     unsigned char *ws;
     int32_t n_buf;
     int prefilled;
+    int codes_map_ready;
 };
 
 namespace {
@@ -180,6 +184,7 @@ lq_status lq_state_create(const lq_config *cfg, void *d_workspace, size_t bytes,
     h->ws = static_cast<unsigned char *>(d_workspace);
     h->n_buf = 0;
     h->prefilled = 0;
+    h->codes_map_ready = 0;
     *out = h;
     return LQ_OK;
 }
@@ -237,10 +242,17 @@ lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, const vo
     if (!h->prefilled) return fail(LQ_ERR_STATE, "decode before lq_prefill_state");
     if (c.mode == LQ_MODE_WINDOW && h->n_buf >= c.window)
         return fail(LQ_ERR_WINDOW_FULL, "window holds W tokens: call lq_window_flush first");
+    if (c.mode == LQ_MODE_WINDOW && !h->codes_map_ready) {
+        cudaError_t e = lq::make_codes_map(&h->codes_map, reinterpret_cast<const int8_t *>(h->ws + h->lay.codes),
+                                           c.d_k, c.batch * c.heads);
+        if (e != cudaSuccess) return cuda_fail(e, "encoding the tensor map of the codes");
+        h->codes_map_ready = 1;
+    }
     lq::DecodeArgs a;
     a.w = views(h);
     a.q = d_q; a.k = d_k; a.v = d_v; a.g = d_g; a.beta = d_beta; a.o = d_o;
     a.n_buf = h->n_buf;
+    a.codes_map = &h->codes_map;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (c.mode == LQ_MODE_WINDOW) e = lq::launch_decode_window(a, c.d_k, c.gate, c.in_dtype, s);

@@ -17,17 +17,28 @@
 // buffer.  It writes no state.
 //
 // Persistent and warp-specialized: four CTAs per SM walk the (sequence, head)
-// units.  In each CTA one producer thread streams every unit's data with 1-D
-// bulk async copies through a ring of three 16 KB shared-memory slots -- a
-// meta segment (row scales, smoothing factors, q/k/v, gate, compensators), the
-// INT8 tile, then the buffered entries in chunks of up to 16 -- and four
-// consumer warps compute.  Each slot has a full mbarrier (bytes landed) and an
-// empty mbarrier that every consumer thread arrives on after its last read,
-// so no block-wide barrier is spent on releasing slots; the consumers meet at
-// one barrier after the operand prep and one per chunk.  The INT8 tile is
-// widened with an exact exponent-bias trick and accumulated with packed FP32
-// FMAs.  Every wait is bounded; an expired wait records LQ_DEVERR_TIMEOUT and
-// all consumer warps leave together at their next barrier.
+// units.  In each CTA one producer thread streams every unit's data through a
+// ring of three 16 KB shared-memory slots -- a meta segment (row scales,
+// smoothing factors, q/k/v, gate, compensators) by 1-D bulk async copies, the
+// INT8 tile by a 2-D tensor copy with 128-byte swizzle, then the buffered
+// entries in chunks of up to 16 -- and four consumer warps compute.  Each
+// slot has a full mbarrier (bytes landed) and an empty mbarrier that every
+// consumer thread arrives on after its last read, so no block-wide barrier is
+// spent on releasing slots; the consumers meet at one barrier after the
+// operand prep and one per chunk.
+//
+// The INT8 pass is an exact integer dot product on the tensor cores.  Each
+// 32-column block of y^q = s*x^q and y^k = s*x^k is written as
+// y = 2^E (d_0 + d_1 2^-7 + d_2 2^-14 + d_3 2^-21) with int8 digits d_p and a
+// block exponent E (every step exact in FP32; the dropped remainder is below
+// 2^-27 of the block maximum).  mma.sync m16n8k32 s8 x s8 -> s32 then forms
+// Q d_p for all 8 (vector, digit) columns at once with exact int32 sums, and
+// the digits are recombined in FP32.  No per-byte widening is needed.
+// Every wait is bounded; an expired wait records LQ_DEVERR_TIMEOUT and all
+// consumer warps leave together at their next barrier.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "lq_kernels.h"
 
 namespace lq {
@@ -53,19 +64,19 @@ struct Shape {
     static constexpr int E = E0 < kPer * kConsumerWarps ? E0 : kPer * kConsumerWarps;
     static constexpr int C_KEY = 4 * D * E;                        // chunk: deltas, keys, omega_j
     static constexpr int C_GATE = C_KEY + KB * D * E;
-    static constexpr int LPR = D / 16;                             // lanes per INT8 row
-    static constexpr int RPW = 32 / LPR;                           // rows per warp per round
-    static constexpr int ROUNDS = D / (kConsumerWarps * RPW);
-    static constexpr int BATCH = ROUNDS < 4 ? ROUNDS : 4;          // rounds loaded together
+    static constexpr int KBLK = D / 32;                            // 32-column blocks (one per prep warp)
+    static constexpr int MT = D / 16 / kConsumerWarps;             // 16-row m-tiles per warp
     static constexpr int VPL = D / 32;                             // key elements per lane
-    // consumer scratch after the ring, in floats
-    static constexpr int S_Y = 0;                  // D/2 float4: (yq pair, yk pair), swizzled
-    static constexpr int S_XQ = 2 * D, S_XK = 3 * D, S_QR = 4 * D, S_KR = 5 * D, S_A = 6 * D, S_B = 7 * D;
-    static constexpr int S_CF = 8 * D;             // 2 x 16 float2 coefficients (double buffer)
-    static constexpr int S_RCK = S_CF + 64, S_RCQ = S_RCK + 8, S_RED = S_RCQ + 8, S_FLOATS = S_RED + 8;
-    static constexpr int SMEM = 128 + kSlots * kSlotBytes + 4 * S_FLOATS;
+    // consumer scratch, in floats: digits (8 x D int8), block scales, vectors,
+    // products, coefficients (two buffers), compensator dots, reductions
+    static constexpr int S_B8 = 0, S_EXP = 2 * D, S_XQ = S_EXP + 8, S_XK = S_XQ + D, S_QR = S_XK + D,
+                         S_KR = S_QR + D, S_A = S_KR + D, S_B = S_A + D, S_CF = S_B + D, S_RCK = S_CF + 64,
+                         S_RCQ = S_RCK + 8, S_RED = S_RCQ + 8, S_FLOATS = S_RED + 8;
+    static constexpr int OFF_BARS = 4 * S_FLOATS;                  // then the ring, 1024-aligned
+    static constexpr int OFF_RING = align_up(OFF_BARS + 16 * kSlots, 1024);
+    static constexpr int SMEM = OFF_RING + kSlots * kSlotBytes + 1024;   // + alignment slack
     static_assert(E >= 4 && E <= kPer * kConsumerWarps, "chunk size");
-    static_assert(ROUNDS % BATCH == 0, "row rounds");
+    static_assert(MT >= 1, "m-tiles");
 };
 
 // Offsets inside a meta segment.
@@ -147,33 +158,82 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Two int8 codes (bytes of word u, already offset by 128) as exact floats.
-__device__ __forceinline__ float2 i8pair(uint32_t u, uint32_t sel_lo, uint32_t sel_hi) {
-    const float2 biased = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, sel_lo)),
-                                      __uint_as_float(__byte_perm(u, 0x4B000000u, sel_hi)));
-    return __fadd2_rn(biased, make_float2(-8388736.0f, -8388736.0f));   // minus (2^23 + 128)
+// Byte offset of the 16-byte chunk `chunk` of row `row` in a D x D int8 tile
+// written by the tensor copy with the 128-byte (D = 128) or 64-byte (D = 64)
+// swizzle: the chunk index is XORed with address bits 7-9 (resp. 7-8).
+template <int D>
+__device__ __forceinline__ int swz(int row, int chunk) {
+    if constexpr (D == 128) return row * 128 + ((chunk ^ (row & 7)) << 4);
+    else return row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4);
 }
 
-// Swizzled slot of the float4 (yq[2m..2m+1], yk[2m..2m+1]) of column block cb:
-// lanes of one quarter-warp read different banks.
-__device__ __forceinline__ int y_slot(int cb, int m) { return cb * 8 + ((m + cb) & 7); }
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
 
+// D (16x8 s32) += A (16x32 s8, row) * B (32x8 s8, col)
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                       uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 2-D tensor copy of the (x, y) box of `map` into shared memory.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 2^k as a float, for |k| <= 126.
+__device__ __forceinline__ float pow2i(int k) { return __int_as_float((127 + k) << 23); }
+
+// Block exponent of a block with maximum |y| = m: 2^E with m 2^-E in [32, 64),
+// returned as (2^-E, 2^E); (0, 0) for a block too small to matter.
+__device__ __forceinline__ float2 block_scale(float m) {
+    const int biased = (__float_as_int(m) >> 23) & 0xff;     // m = 1.f x 2^(biased - 127)
+    if (biased < 20) return make_float2(0.0f, 0.0f);          // |y| < 2^-107 (or zero)
+    const int E = biased - 127 + 1 - 6;
+    return make_float2(pow2i(-E), pow2i(E));
+}
+
+// The four base-2^7 int8 digits of y * 2^-E (|y 2^-E| < 64), packed low to high.
+__device__ __forceinline__ uint32_t digits4(float y, float down) {
+    float r = y * down;
+    uint32_t out = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float d = rintf(r);
+        out |= ((uint32_t)(int)d & 0xffu) << (8 * p);
+        r = (r - d) * 128.0f;
+    }
+    return out;
+}
 template <int D, bool KDA, typename InT, typename KeyT>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_window_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    decode_window_kernel(DecodeArgs a, const __grid_constant__ CUtensorMap codes_map) {
     using Sh = Shape<D, KDA, InT, KeyT>;
-    constexpr int E = Sh::E, LPR = Sh::LPR, RPW = Sh::RPW, ROUNDS = Sh::ROUNDS, BATCH = Sh::BATCH;
-    constexpr int VPL = Sh::VPL;
+    constexpr int E = Sh::E, KBLK = Sh::KBLK, MT = Sh::MT, VPL = Sh::VPL;
     const Views &w = a.w;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ncr = w.n_comp_rows, ncc = w.n_comp_cols, cis = w.comp_index_stride, ncomp = ncr + ncc;
     const int n_buf = a.n_buf, nchunks = (n_buf + E - 1) / E, units = w.units;
     const Meta M = meta_layout<D, KDA, InT>(ncr, ncc, cis);
 
-    extern __shared__ __align__(128) unsigned char sm[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm);
+    extern __shared__ __align__(1024) unsigned char sm_raw[];
+    // the swizzled tensor copies need a 1024-byte aligned destination
+    unsigned char *sm = sm_raw + ((1024 - (smem_u32(sm_raw) & 1023)) & 1023);
+    float *scr = reinterpret_cast<float *>(sm);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + Sh::OFF_BARS);
     uint64_t *empty = full + kSlots;
-    unsigned char *ring = sm + 128;
-    float *scr = reinterpret_cast<float *>(ring + kSlots * kSlotBytes);
+    unsigned char *ring = sm + Sh::OFF_RING;
 
     if (tid == 0) {
         for (int i = 0; i < kSlots; ++i) {
@@ -187,7 +247,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_window_kernel(Dec
     // ================================================================ producer
     if (warp == kConsumerWarps) {
         if (lane != 0) return;
-        const uint64_t stream_once = l2_policy_evict_first();
         const uint32_t in_b = (uint32_t)sizeof(InT) * D;
         int slot = 0;
         uint32_t ph = 0;
@@ -225,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_window_kernel(Dec
             if (dst == nullptr) return;
             bar = &full[slot];
             mbar_arrive_expect_tx(bar, D * D);
-            bulk_g2s_stream(dst, w.codes + (size_t)u * D * D, D * D, bar, stream_once);
+            tma_load_2d(dst, &codes_map, 0, u * D, bar);
             advance();
             for (int c = 0; c < nchunks; ++c) {
                 dst = acquire(u, -3 - c);
@@ -246,7 +305,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_window_kernel(Dec
     }
 
     // =============================================================== consumers
-    float4 *sY = reinterpret_cast<float4 *>(scr + Sh::S_Y);
+    int8_t *sB8 = reinterpret_cast<int8_t *>(scr + Sh::S_B8);   // [8][D] digits: y^q d_0..3, y^k d_0..3
+    float *sExp = scr + Sh::S_EXP;                              // 2^E per (vector, 32-column block)
     float *sXq = scr + Sh::S_XQ, *sXk = scr + Sh::S_XK, *sQr = scr + Sh::S_QR, *sKr = scr + Sh::S_KR;
     float *sA = scr + Sh::S_A, *sB = scr + Sh::S_B;
     float2 *sCf = reinterpret_cast<float2 *>(scr + Sh::S_CF);
@@ -300,9 +360,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_window_kernel(Dec
             sXk[j] = xk;
             sQr[j] = qj;
             sKr[j] = kj;
-            float *yf = reinterpret_cast<float *>(sY + y_slot(j >> 4, (j & 15) >> 1));
-            yf[j & 1] = sj * xq;
-            yf[2 + (j & 1)] = sj * xk;
+            // exact int8 digits of y^q_j and y^k_j with this warp's block exponents
+            const float yq = sj * xq, yk = sj * xk;
+            const float2 eq = block_scale(group_max<32>(fabsf(yq)));
+            const float2 ek = block_scale(group_max<32>(fabsf(yk)));
+            const uint32_t dq = digits4(yq, eq.x), dk = digits4(yk, ek.x);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                sB8[p * D + j] = (int8_t)((dq >> (8 * p)) & 0xff);
+                sB8[(4 + p) * D + j] = (int8_t)((dk >> (8 * p)) & 0xff);
+            }
+            if (lane == 0) {
+                sExp[warp] = eq.y;
+                sExp[4 + warp] = ek.y;
+            }
             kq = kj * qj;
             if (KDA) {
                 if (fabs(G_j) > kMaxAbsGateSum) report_error(w.err, LQ_DEVERR_RANGE, u, j);
@@ -355,47 +426,45 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_window_kernel(Dec
         load_vec<VPL>((KDA ? sXq : sQr) + lane * VPL, xs_q);
 
         // ---------------------------- A2: one pass over the INT8 tile
+        // a_i = sigma_i sum_j Q_ij y^q_j and b_i = sigma_i sum_j Q_ij y^k_j, as
+        // exact int8 products on the tensor cores (see the file comment)
         bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
         {
-            const int8_t *sQ = reinterpret_cast<const int8_t *>(ring + slot * kSlotBytes);
+            const unsigned char *tile = ring + slot * kSlotBytes;
             const float *sSig = reinterpret_cast<const float *>(mp + M.sig);
-            const int cb = lane % LPR, rsub = lane / LPR;
-            float2 yq[8], yk[8];
+            const int g = lane >> 2, c4 = lane & 3;
+            uint32_t bf[KBLK][2];                  // B fragments: digit column g, k = 4*c4 (+16)
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const float4 t = sY[y_slot(cb, m)];
-                yq[m] = make_float2(t.x, t.y);
-                yk[m] = make_float2(t.z, t.w);
+            for (int kb = 0; kb < KBLK; ++kb) {
+                bf[kb][0] = *reinterpret_cast<const uint32_t *>(sB8 + g * D + kb * 32 + 4 * c4);
+                bf[kb][1] = *reinterpret_cast<const uint32_t *>(sB8 + g * D + kb * 32 + 16 + 4 * c4);
             }
+            // this lane's digit columns: 2*c4 and 2*c4+1, i.e. vector c4/2, digits 2*(c4&1) and +1
+            const float w0 = (c4 & 1) ? 0x1p-14f : 1.0f, w1 = w0 * 0x1p-7f;
+            float scale[KBLK];
 #pragma unroll
-            for (int r0 = 0; r0 < ROUNDS; r0 += BATCH) {
-                uint4 qw[BATCH];
+            for (int kb = 0; kb < KBLK; ++kb) scale[kb] = sExp[(c4 >> 1) * 4 + kb];
+            const uint32_t tile_s = smem_u32(tile);
+            const int q = lane >> 3, rr = lane & 7;   // ldmatrix: matrix q, row rr within it
 #pragma unroll
-                for (int r = 0; r < BATCH; ++r) {
-                    const int i = (r0 + r) * (kConsumerWarps * RPW) + warp * RPW + rsub;
-                    qw[r] = *reinterpret_cast<const uint4 *>(sQ + i * D + cb * 16);
+            for (int mt = 0; mt < MT; ++mt) {
+                const int m0 = (warp * MT + mt) * 16;
+                float v0 = 0.0f, v1 = 0.0f;        // rows m0 + g and m0 + g + 8
+#pragma unroll
+                for (int kb = 0; kb < KBLK; ++kb) {
+                    uint32_t a0, a1, a2, a3;
+                    ldmatrix_x4(tile_s + swz<D>(m0 + (q & 1) * 8 + rr, kb * 2 + (q >> 1)), a0, a1, a2, a3);
+                    int acc4[4] = {0, 0, 0, 0};
+                    mma_s8(acc4, a0, a1, a2, a3, bf[kb][0], bf[kb][1]);
+                    v0 = fmaf(scale[kb], fmaf((float)acc4[1], w1, (float)acc4[0] * w0), v0);
+                    v1 = fmaf(scale[kb], fmaf((float)acc4[3], w1, (float)acc4[2] * w0), v1);
                 }
-#pragma unroll
-                for (int r = 0; r < BATCH; ++r) {
-                    const int i = (r0 + r) * (kConsumerWarps * RPW) + warp * RPW + rsub;
-                    const uint32_t words[4] = {qw[r].x ^ 0x80808080u, qw[r].y ^ 0x80808080u,
-                                               qw[r].z ^ 0x80808080u, qw[r].w ^ 0x80808080u};
-                    float2 pa = make_float2(0.0f, 0.0f), pb = make_float2(0.0f, 0.0f);
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const float2 f01 = i8pair(words[h], 0x7540, 0x7541);
-                        const float2 f23 = i8pair(words[h], 0x7542, 0x7543);
-                        pa = __ffma2_rn(f01, yq[2 * h], pa);
-                        pb = __ffma2_rn(f01, yk[2 * h], pb);
-                        pa = __ffma2_rn(f23, yq[2 * h + 1], pa);
-                        pb = __ffma2_rn(f23, yk[2 * h + 1], pb);
-                    }
-                    const float sa = group_sum<LPR>(pa.x + pa.y);
-                    const float sb = group_sum<LPR>(pb.x + pb.y);
-                    if (cb == 0) {
-                        sA[i] = sSig[i] * sa;
-                        sB[i] = sSig[i] * sb;
-                    }
+                v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+                v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+                if ((c4 & 1) == 0) {
+                    float *dst = (c4 == 0) ? sA : sB;
+                    dst[m0 + g] = sSig[m0 + g] * v0;
+                    dst[m0 + g + 8] = sSig[m0 + g + 8] * v1;
                 }
             }
         }
@@ -547,11 +616,32 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
         if (dev >= 0 && dev < 64) opted_in[dev] = true;
     }
     const int grid = min(a.w.units, kCtasPerSm * sm_count());
-    kern<<<grid, kThreads, Sh::SMEM, s>>>(a);
+    kern<<<grid, kThreads, Sh::SMEM, s>>>(a, *reinterpret_cast<const CUtensorMap *>(a.codes_map));
     return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t make_codes_map(void *map_out, const int8_t *codes, int d, int units) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (encode == nullptr) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorNotSupported;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)units * (cuuint64_t)d};
+    const cuuint64_t strides[1] = {(cuuint64_t)d};
+    const cuuint32_t box[2] = {(cuuint32_t)d, (cuuint32_t)d};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(reinterpret_cast<CUtensorMap *>(map_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                              const_cast<int8_t *>(codes), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
 
 cudaError_t launch_decode_window(const DecodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s) {
     const bool kda = (gate == LQ_GATE_CHANNEL);

@@ -28,7 +28,12 @@ struct DecodeArgs {
     const float *beta;
     float *o;
     int n_buf;         // tokens buffered before this one (windowed mode)
+    const void *codes_map;   // host copy of the tensor map of the INT8 codes (windowed mode)
 };
+
+// Encode the tensor map the windowed decode uses to load one unit's INT8 tile
+// (d x d, 128- or 64-byte swizzle) from `codes` ([units][d][d]).  Host only.
+cudaError_t make_codes_map(void *map_out, const int8_t *codes, int d, int units);
 
 // d = d_k = d_v in {64, 128}; gate: LQ_GATE_*; in_dtype: LQ_DTYPE_*.
 cudaError_t launch_encode(const EncodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
