@@ -69,9 +69,10 @@ struct Shape {
     static constexpr int VPL = D / 32;                             // key elements per lane
     // consumer scratch, in floats: digits (8 x D int8), block scales, vectors,
     // products, coefficients (two buffers), compensator dots, reductions
+    static constexpr int RED = 1 + 2 * 8;                          // kq, then (k, q) dots of 8 row comps
     static constexpr int S_B8 = 0, S_EXP = 2 * D, S_XQ = S_EXP + 8, S_XK = S_XQ + D, S_QR = S_XK + D,
-                         S_KR = S_QR + D, S_A = S_KR + D, S_B = S_A + D, S_CF = S_B + D, S_RCK = S_CF + 64,
-                         S_RCQ = S_RCK + 8, S_RED = S_RCQ + 8, S_FLOATS = S_RED + 8;
+                         S_KR = S_QR + D, S_A = S_KR + D, S_B = S_A + D, S_CF = S_B + D,
+                         S_RED = S_CF + 64, S_FLOATS = S_RED + kConsumerWarps * RED;
     static constexpr int OFF_BARS = 4 * S_FLOATS;                  // then the ring, 1024-aligned
     static constexpr int OFF_RING = align_up(OFF_BARS + 16 * kSlots, 1024);
     static constexpr int SMEM = OFF_RING + kSlots * kSlotBytes + 1024;   // + alignment slack
@@ -310,8 +311,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     float *sXq = scr + Sh::S_XQ, *sXk = scr + Sh::S_XK, *sQr = scr + Sh::S_QR, *sKr = scr + Sh::S_KR;
     float *sA = scr + Sh::S_A, *sB = scr + Sh::S_B;
     float2 *sCf = reinterpret_cast<float2 *>(scr + Sh::S_CF);
-    float *sRck = scr + Sh::S_RCK, *sRcq = scr + Sh::S_RCQ, *sRed = scr + Sh::S_RED;
+    float *sRed = scr + Sh::S_RED;                              // [warp][kq, row-comp dots]
     const bool owns_row = tid < D;                 // thread i: state row i and key channel i
+    constexpr int CPL = D / 8;                     // key channels per lane in the entry dots
+    // entry dots: 8 lanes per entry; lane s covers channels 32m + 4s + t (m < D/32, t < 4)
+    const int dot_s = lane & 7, dot_e = warp * 4 + (lane >> 3);
 
     int slot = 0;
     uint32_t ph = 0;
@@ -319,15 +323,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if (++slot == kSlots) { slot = 0; ph ^= 1u; }
     };
     int u = blockIdx.x;
-    float beta_n = 0.0f, g_n = 0.0f;
+    float beta_n = 0.0f, g_n = 0.0f, gam_n = 0.0f;
     double G_n = 0.0;
     if (u < units) {
         beta_n = a.beta[u];
-        if (!KDA) { g_n = a.g[u]; G_n = w.gate_sum[u]; }
+        if (!KDA) {
+            g_n = a.g[u];
+            G_n = w.gate_sum[u] + (double)g_n;
+            gam_n = exp_of_double(G_n);
+        }
     }
     for (; u < units; u += gridDim.x) {
         const float beta = beta_n;
-        const double Gs = KDA ? 0.0 : G_n + (double)g_n;   // scalar gate: G_t
+        const double Gs = G_n;                     // scalar gate: G_t
+        const float gam_s = gam_n;                 // scalar gate: gamma_t
         const int un = u + gridDim.x;
         if (un < units) {                          // next unit's scalars, in flight meanwhile
             beta_n = a.beta[un];
@@ -340,8 +349,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const int meta_slot = slot;
         advance();
         double G_j = 0.0;
-        float key_out = 0.0f, v_i = 0.0f, kq = 0.0f, gam_s = 0.0f;
-        if (!KDA) gam_s = exp_of_double(Gs);
+        float key_out = 0.0f, v_i = 0.0f;
         if (owns_row) {
             const int j = tid;
             float gam;
@@ -374,7 +382,44 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 sExp[warp] = eq.y;
                 sExp[4 + warp] = ek.y;
             }
-            kq = kj * qj;
+            // k_t . q_t and the row compensators' dots k_c . x, reduced per warp
+            // (compensator rows 0..3 together with k.q; rows 4..7, when used, after)
+            {
+                const float *crow = reinterpret_cast<const float *>(mp + M.crow);
+                float part[9];
+                part[0] = kj * qj;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float kc = (c < ncr) ? crow[c * D + j] : 0.0f;
+                    part[1 + 2 * c] = kc * xk;
+                    part[2 + 2 * c] = kc * xq;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                    for (int i = 0; i < 9; ++i) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
+                if (lane == 0) {
+#pragma unroll
+                    for (int i = 0; i < 9; ++i) sRed[warp * Sh::RED + i] = part[i];
+                }
+                if (ncr > 4) {
+                    float more[8];
+#pragma unroll
+                    for (int c = 4; c < 8; ++c) {
+                        const float kc = (c < ncr) ? crow[c * D + j] : 0.0f;
+                        more[2 * (c - 4)] = kc * xk;
+                        more[2 * (c - 4) + 1] = kc * xq;
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) more[i] += __shfl_xor_sync(0xffffffffu, more[i], o);
+                    if (lane == 0) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) sRed[warp * Sh::RED + 9 + i] = more[i];
+                    }
+                }
+            }
             if (KDA) {
                 if (fabs(G_j) > kMaxAbsGateSum) report_error(w.err, LQ_DEVERR_RANGE, u, j);
                 key_out = kj * exp_of_double(-G_j);          // kappa_j
@@ -383,35 +428,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
         }
         if (!KDA && tid == 0 && fabs(Gs) > kMaxAbsGateSum) report_error(w.err, LQ_DEVERR_RANGE, u, -1);
-        kq = group_sum<32>(kq);
-        if (lane == 0) sRed[warp] = kq;
         if (consumer_sync_or(bad)) {
             if (tid == 0) report_error(w.err, LQ_DEVERR_TIMEOUT, u, 0);
             return;
         }
-        kq = 0.0f;
-#pragma unroll
-        for (int i = 0; i < kConsumerWarps; ++i) kq += sRed[i];
 
-        // compensators: row ones as dots k_c . x (one warp each), column ones per row
-        for (int c = warp; c < ncr; c += kConsumerWarps) {
-            const float *kc = reinterpret_cast<const float *>(mp + M.crow) + c * D;
-            float dk = 0.0f, dq = 0.0f;
-            for (int j = lane; j < D; j += 32) {
-                dk = fmaf(kc[j], sXk[j], dk);
-                dq = fmaf(kc[j], sXq[j], dq);
-            }
-            dk = group_sum<32>(dk);
-            dq = group_sum<32>(dq);
-            if (lane == 0) { sRck[c] = dk; sRcq[c] = dq; }
-        }
-        float2 acc = make_float2(0.0f, 0.0f);      // (S_{t-1} x^k, S_{t-1} x^q) contributions of this row
-        int comp_row = -1;
+        // kq, this row's compensator contributions (row and column ones)
+        float kq = 0.0f;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) kq += sRed[i * Sh::RED];
+        float2 acc = make_float2(0.0f, 0.0f);      // (S_{t-1} x^k, S_{t-1} x^q) parts of this row
         if (owns_row && ncomp > 0) {
             const int32_t *cidx = reinterpret_cast<const int32_t *>(mp + M.cidx);
             const float *ccol = reinterpret_cast<const float *>(mp + M.ccol);
-            for (int c = 0; c < ncr; ++c)
-                if (cidx[c] == tid) comp_row = c;
+            for (int c = 0; c < ncr; ++c) {
+                if (cidx[c] == tid) {
+#pragma unroll
+                    for (int i = 0; i < D / 32; ++i) {
+                        acc.x += sRed[i * Sh::RED + 1 + 2 * c];
+                        acc.y += sRed[i * Sh::RED + 2 + 2 * c];
+                    }
+                }
+            }
             for (int c = 0; c < ncc; ++c) {
                 const int j = cidx[ncr + c];
                 const float vc = ccol[c * D + tid];
@@ -419,11 +457,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 acc.y = fmaf(vc, sXq[j], acc.y);
             }
         }
-
-        // entry-dot operands: this lane's slice of (k_t, q_t) or (x^k, x^q)
-        float xs_k[VPL], xs_q[VPL];
-        load_vec<VPL>((KDA ? sXk : sKr) + lane * VPL, xs_k);
-        load_vec<VPL>((KDA ? sXq : sQr) + lane * VPL, xs_q);
 
         // ---------------------------- A2: one pass over the INT8 tile
         // a_i = sigma_i sum_j Q_ij y^q_j and b_i = sigma_i sum_j Q_ij y^k_j, as
@@ -446,16 +479,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             for (int kb = 0; kb < KBLK; ++kb) scale[kb] = sExp[(c4 >> 1) * 4 + kb];
             const uint32_t tile_s = smem_u32(tile);
             const int q = lane >> 3, rr = lane & 7;   // ldmatrix: matrix q, row rr within it
+            uint32_t af[MT][KBLK][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int kb = 0; kb < KBLK; ++kb)
+                    ldmatrix_x4(tile_s + swz<D>((warp * MT + mt) * 16 + (q & 1) * 8 + rr, kb * 2 + (q >> 1)),
+                                af[mt][kb][0], af[mt][kb][1], af[mt][kb][2], af[mt][kb][3]);
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 const int m0 = (warp * MT + mt) * 16;
                 float v0 = 0.0f, v1 = 0.0f;        // rows m0 + g and m0 + g + 8
 #pragma unroll
                 for (int kb = 0; kb < KBLK; ++kb) {
-                    uint32_t a0, a1, a2, a3;
-                    ldmatrix_x4(tile_s + swz<D>(m0 + (q & 1) * 8 + rr, kb * 2 + (q >> 1)), a0, a1, a2, a3);
                     int acc4[4] = {0, 0, 0, 0};
-                    mma_s8(acc4, a0, a1, a2, a3, bf[kb][0], bf[kb][1]);
+                    mma_s8(acc4, af[mt][kb][0], af[mt][kb][1], af[mt][kb][2], af[mt][kb][3], bf[kb][0], bf[kb][1]);
                     v0 = fmaf(scale[kb], fmaf((float)acc4[1], w1, (float)acc4[0] * w0), v0);
                     v1 = fmaf(scale[kb], fmaf((float)acc4[3], w1, (float)acc4[2] * w0), v1);
                 }
@@ -481,55 +519,33 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const float *sOmega = reinterpret_cast<const float *>(cp + Sh::C_GATE);
             const int ne = min(E, n_buf - c * E);
             float2 *cf = sCf + (c & 1) * 16;
-            // dots of this warp's entries with (x^k, x^q): v[0..3] for x^k, v[4..7] for x^q
-            float v[2 * kPer];
-#pragma unroll
-            for (int r = 0; r < kPer; ++r) {
-                const int el = warp + r * kConsumerWarps;
-                float dk = 0.0f, dq = 0.0f;
-                if (el < ne) {
-                    float kv[VPL];
-                    load_key<KeyT, VPL>(sKey + el * D + lane * VPL, kv);
-#pragma unroll
-                    for (int t = 0; t < VPL; ++t) {
-                        dk = fmaf(kv[t], xs_k[t], dk);
-                        dq = fmaf(kv[t], xs_q[t], dq);
-                    }
-                }
-                v[r] = dk;
-                v[kPer + r] = dq;
-            }
-            // butterfly reduce-scatter of the 8 partial sums over the warp: lane l
-            // ends with the total of value 4*b4 + 2*b3 + b2 (b = bits of l)
+            // coefficients kappa_e . (x^k, x^q): 8 lanes per entry, 3-level reduction;
+            // every lane takes part in the shuffles, lanes past the chunk with zeros
             {
-                const bool hi16 = lane & 16, hi8 = lane & 8, hi4 = lane & 4;
-                float h4[4];
+                const bool live_e = dot_e < ne;
+                const float *xk = KDA ? sXk : sKr, *xq = KDA ? sXq : sQr;
+                float dk0 = 0.0f, dk1 = 0.0f, dq0 = 0.0f, dq1 = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float send = hi16 ? v[i] : v[i + 4];
-                    const float keep = hi16 ? v[i + 4] : v[i];
-                    h4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                for (int m = 0; m < D / 32 && live_e; ++m) {
+                    const int j0 = 32 * m + 4 * dot_s;
+                    float kv[4];
+                    load_key<KeyT, 4>(sKey + dot_e * D + j0, kv);
+                    const float4 a4 = *reinterpret_cast<const float4 *>(xk + j0);
+                    const float4 b4 = *reinterpret_cast<const float4 *>(xq + j0);
+                    dk0 = fmaf(kv[0], a4.x, dk0); dk1 = fmaf(kv[1], a4.y, dk1);
+                    dk0 = fmaf(kv[2], a4.z, dk0); dk1 = fmaf(kv[3], a4.w, dk1);
+                    dq0 = fmaf(kv[0], b4.x, dq0); dq1 = fmaf(kv[1], b4.y, dq1);
+                    dq0 = fmaf(kv[2], b4.z, dq0); dq1 = fmaf(kv[3], b4.w, dq1);
                 }
-                float h2[2];
+                float dk = dk0 + dk1, dq = dq0 + dq1;
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const float send = hi8 ? h4[i] : h4[i + 2];
-                    const float keep = hi8 ? h4[i + 2] : h4[i];
-                    h2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                for (int o = 4; o > 0; o >>= 1) {
+                    dk += __shfl_xor_sync(0xffffffffu, dk, o);
+                    dq += __shfl_xor_sync(0xffffffffu, dq, o);
                 }
-                float s1;
-                {
-                    const float send = hi4 ? h2[0] : h2[1];
-                    const float keep = hi4 ? h2[1] : h2[0];
-                    s1 = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-                }
-                s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-                s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-                const int r = (hi8 ? 2 : 0) + (hi4 ? 1 : 0);
-                const int el = warp + r * kConsumerWarps;
-                if ((lane & 3) == 0 && el < ne) {
-                    const float f = KDA ? 1.0f : gam_s * sOmega[el];
-                    reinterpret_cast<float *>(cf + el)[hi16 ? 1 : 0] = f * s1;
+                if (live_e && dot_s == 0) {
+                    const float f = KDA ? 1.0f : gam_s * sOmega[dot_e];
+                    cf[dot_e] = make_float2(f * dk, f * dq);
                 }
             }
             if (consumer_sync_or(bad)) {
@@ -537,19 +553,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 return;
             }
             if (owns_row) {
-                float2 acc2 = make_float2(0.0f, 0.0f);
-                int el = 0;
-                for (; el + 1 < ne; el += 2) {
-                    const float d0 = sDelta[el * D + tid], d1 = sDelta[(el + 1) * D + tid];
-                    acc = __ffma2_rn(make_float2(d0, d0), cf[el], acc);
-                    acc2 = __ffma2_rn(make_float2(d1, d1), cf[el + 1], acc2);
+                float2 p[4] = {acc, make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+#pragma unroll
+                for (int el = 0; el < E; ++el) {
+                    const bool live = el < ne;
+                    const float d0 = live ? sDelta[el * D + tid] : 0.0f;
+                    const float2 cc = live ? cf[el] : make_float2(0.0f, 0.0f);
+                    p[el & 3] = __ffma2_rn(make_float2(d0, d0), cc, p[el & 3]);
                 }
-                if (el < ne) {
-                    const float d0 = sDelta[el * D + tid];
-                    acc = __ffma2_rn(make_float2(d0, d0), cf[el], acc);
-                }
-                acc.x += acc2.x;
-                acc.y += acc2.y;
+                acc.x = (p[0].x + p[1].x) + (p[2].x + p[3].x);
+                acc.y = (p[0].y + p[1].y) + (p[2].y + p[3].y);
             }
             mbar_arrive(&empty[slot]);             // done with this chunk
             advance();
@@ -562,11 +575,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // ------------------------------------------------ A4: emit and append
         if (owns_row) {
             const int i = tid;
-            float sk = acc.x + sB[i], so = acc.y + sA[i];
-            if (comp_row >= 0) {
-                sk += sRck[comp_row];
-                so += sRcq[comp_row];
-            }
+            const float sk = acc.x + sB[i], so = acc.y + sA[i];
             const float delta = beta * (v_i - sk);
             const size_t slot_g = (size_t)u * w.window + n_buf;
             a.o[(size_t)u * D + i] = fmaf(delta, kq, so);
@@ -581,6 +590,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if (!KDA && tid == 0) {
             w.buf_gate[(size_t)u * w.window_pad + n_buf] = exp_of_double(-Gs);
             w.gate_sum[u] = Gs;
+        }
+        if (!KDA && un < units) {                  // next unit's G_t and gamma_t, off its critical path
+            G_n = G_n + (double)g_n;
+            gam_n = exp_of_double(G_n);
         }
     }
 }
