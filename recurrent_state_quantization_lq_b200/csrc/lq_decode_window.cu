@@ -66,7 +66,6 @@ struct Shape {
     static constexpr int C_GATE = C_KEY + KB * D * E;
     static constexpr int KBLK = D / 32;                            // 32-column blocks (one per prep warp)
     static constexpr int MT = D / 16 / kConsumerWarps;             // 16-row m-tiles per warp
-    static constexpr int VPL = D / 32;                             // key elements per lane
     // consumer scratch, in floats: digits (8 x D int8), block scales, vectors,
     // products, coefficients (two buffers), compensator dots, reductions
     static constexpr int RED = 1 + 2 * 8;                          // kq, then (k, q) dots of 8 row comps
@@ -130,17 +129,6 @@ __device__ __forceinline__ void load_key(const KeyT *p, float (&out)[VPL]) {
     }
 }
 
-template <int VPL>
-__device__ __forceinline__ void load_vec(const float *p, float (&out)[VPL]) {
-    if constexpr (VPL == 4) {
-        float4 w = *reinterpret_cast<const float4 *>(p);
-        out[0] = w.x; out[1] = w.y; out[2] = w.z; out[3] = w.w;
-    } else {
-        float2 w = *reinterpret_cast<const float2 *>(p);
-        out[0] = w.x; out[1] = w.y;
-    }
-}
-
 // Consumer barrier that also ORs a predicate over the consumer threads.
 __device__ __forceinline__ bool consumer_sync_or(bool pred) {
     uint32_t r;
@@ -193,6 +181,10 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// Exact int -> float for |x| < 2^22 without the conversion unit: at 1.5 * 2^23
+// the float spacing is 1, so the word 0x4B400000 + x is the number 1.5 * 2^23 + x.
+__device__ __forceinline__ float i2f_exact(int x) { return __int_as_float(0x4B400000 + x) - 12582912.0f; }
+
 // 2^k as a float, for |k| <= 126.
 __device__ __forceinline__ float pow2i(int k) { return __int_as_float((127 + k) << 23); }
 
@@ -221,7 +213,7 @@ template <int D, bool KDA, typename InT, typename KeyT>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_window_kernel(DecodeArgs a, const __grid_constant__ CUtensorMap codes_map) {
     using Sh = Shape<D, KDA, InT, KeyT>;
-    constexpr int E = Sh::E, KBLK = Sh::KBLK, MT = Sh::MT, VPL = Sh::VPL;
+    constexpr int E = Sh::E, KBLK = Sh::KBLK, MT = Sh::MT;
     const Views &w = a.w;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ncr = w.n_comp_rows, ncc = w.n_comp_cols, cis = w.comp_index_stride, ncomp = ncr + ncc;
@@ -313,7 +305,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     float2 *sCf = reinterpret_cast<float2 *>(scr + Sh::S_CF);
     float *sRed = scr + Sh::S_RED;                              // [warp][kq, row-comp dots]
     const bool owns_row = tid < D;                 // thread i: state row i and key channel i
-    constexpr int CPL = D / 8;                     // key channels per lane in the entry dots
     // entry dots: 8 lanes per entry; lane s covers channels 32m + 4s + t (m < D/32, t < 4)
     const int dot_s = lane & 7, dot_e = warp * 4 + (lane >> 3);
 
@@ -370,8 +361,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             sKr[j] = kj;
             // exact int8 digits of y^q_j and y^k_j with this warp's block exponents
             const float yq = sj * xq, yk = sj * xk;
-            const float2 eq = block_scale(group_max<32>(fabsf(yq)));
-            const float2 ek = block_scale(group_max<32>(fabsf(yk)));
+            // non-negative floats order like their bit patterns: one integer max
+            const float2 eq = block_scale(__uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(yq)))));
+            const float2 ek = block_scale(__uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(yk)))));
             const uint32_t dq = digits4(yq, eq.x), dk = digits4(yk, ek.x);
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
@@ -386,22 +378,30 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             // (compensator rows 0..3 together with k.q; rows 4..7, when used, after)
             {
                 const float *crow = reinterpret_cast<const float *>(mp + M.crow);
-                float part[9];
-                part[0] = kj * qj;
+                float kq_p = kj * qj;
+                float v[8];                        // (k_c . x^k, k_c . x^q) of rows c < 4
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const float kc = (c < ncr) ? crow[c * D + j] : 0.0f;
-                    part[1 + 2 * c] = kc * xk;
-                    part[2 + 2 * c] = kc * xq;
+                    v[2 * c] = kc * xk;
+                    v[2 * c + 1] = kc * xq;
                 }
+                // butterfly reduce-scatter: lane l ends with the warp total of value
+                // 4*b4 + 2*b3 + b2 (b = bits of l); k.q by a plain 5-level sum
+                const bool hi16 = lane & 16, hi8 = lane & 8, hi4 = lane & 4;
+                float h4[4], h2[2], s1;
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
+                for (int i = 0; i < 4; ++i)
+                    h4[i] = (hi16 ? v[i + 4] : v[i]) + __shfl_xor_sync(0xffffffffu, hi16 ? v[i] : v[i + 4], 16);
 #pragma unroll
-                    for (int i = 0; i < 9; ++i) part[i] += __shfl_xor_sync(0xffffffffu, part[i], o);
-                if (lane == 0) {
-#pragma unroll
-                    for (int i = 0; i < 9; ++i) sRed[warp * Sh::RED + i] = part[i];
-                }
+                for (int i = 0; i < 2; ++i)
+                    h2[i] = (hi8 ? h4[i + 2] : h4[i]) + __shfl_xor_sync(0xffffffffu, hi8 ? h4[i] : h4[i + 2], 8);
+                s1 = (hi4 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, hi4 ? h2[0] : h2[1], 4);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+                kq_p = group_sum<32>(kq_p);
+                if ((lane & 3) == 0) sRed[warp * Sh::RED + 1 + (hi16 ? 4 : 0) + (hi8 ? 2 : 0) + (hi4 ? 1 : 0)] = s1;
+                if (lane == 0) sRed[warp * Sh::RED] = kq_p;
                 if (ncr > 4) {
                     float more[8];
 #pragma unroll
@@ -439,22 +439,29 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         for (int i = 0; i < D / 32; ++i) kq += sRed[i * Sh::RED];
         float2 acc = make_float2(0.0f, 0.0f);      // (S_{t-1} x^k, S_{t-1} x^q) parts of this row
         if (owns_row && ncomp > 0) {
+            // all index and vector loads first, then the dependent x loads
             const int32_t *cidx = reinterpret_cast<const int32_t *>(mp + M.cidx);
             const float *ccol = reinterpret_cast<const float *>(mp + M.ccol);
-            for (int c = 0; c < ncr; ++c) {
-                if (cidx[c] == tid) {
+            int jc[8], rc = -1;
+            float vcol[8];
 #pragma unroll
-                    for (int i = 0; i < D / 32; ++i) {
-                        acc.x += sRed[i * Sh::RED + 1 + 2 * c];
-                        acc.y += sRed[i * Sh::RED + 2 + 2 * c];
-                    }
-                }
+            for (int c = 0; c < 8; ++c) {
+                const bool on = c < ncc;
+                jc[c] = on ? cidx[ncr + c] : 0;
+                vcol[c] = on ? ccol[c * D + tid] : 0.0f;
+                if (c < ncr && cidx[c] == tid) rc = c;
             }
-            for (int c = 0; c < ncc; ++c) {
-                const int j = cidx[ncr + c];
-                const float vc = ccol[c * D + tid];
-                acc.x = fmaf(vc, sXk[j], acc.x);
-                acc.y = fmaf(vc, sXq[j], acc.y);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                acc.x = fmaf(vcol[c], sXk[jc[c]], acc.x);
+                acc.y = fmaf(vcol[c], sXq[jc[c]], acc.y);
+            }
+            if (rc >= 0) {
+#pragma unroll
+                for (int i = 0; i < D / 32; ++i) {
+                    acc.x += sRed[i * Sh::RED + 1 + 2 * rc];
+                    acc.y += sRed[i * Sh::RED + 2 + 2 * rc];
+                }
             }
         }
 
@@ -494,8 +501,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 for (int kb = 0; kb < KBLK; ++kb) {
                     int acc4[4] = {0, 0, 0, 0};
                     mma_s8(acc4, af[mt][kb][0], af[mt][kb][1], af[mt][kb][2], af[mt][kb][3], bf[kb][0], bf[kb][1]);
-                    v0 = fmaf(scale[kb], fmaf((float)acc4[1], w1, (float)acc4[0] * w0), v0);
-                    v1 = fmaf(scale[kb], fmaf((float)acc4[3], w1, (float)acc4[2] * w0), v1);
+                    v0 = fmaf(scale[kb], fmaf(i2f_exact(acc4[1]), w1, i2f_exact(acc4[0]) * w0), v0);
+                    v1 = fmaf(scale[kb], fmaf(i2f_exact(acc4[3]), w1, i2f_exact(acc4[2]) * w0), v1);
                 }
                 v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
                 v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
