@@ -37,7 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from recurrent_state_quantization_lq_b200 import inputs  # noqa: E402
+from recurrent_state_quantization_lq_b200 import inputs, ranks  # noqa: E402
 
 METRIC = "decode tokens/s per layer & achieved HBM GB/s vs 8 TB/s roofline (INT8 vs FP32 state)"
 UNIT = "tokens/s per layer"
@@ -157,33 +157,21 @@ class ClockSampler:
 # -------------------------------------------------------------- distributed
 
 def dist_setup(n_gpus: int):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = ranks.env_ranks()
     if world > 1:
-        import datetime
-        import torch.distributed as dist
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        ranks.init("nccl", torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
     return rank, world, local
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    ranks.barrier(world)
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return ranks.max_over_ranks(x, world, device=torch.device("cuda", torch.cuda.current_device()))
 
 
 # ------------------------------------------------------------ the CPU oracle
@@ -284,7 +272,7 @@ def run_ours(args, rank, world, local):
     d, kda = wl.d_k, wl.per_channel_gate
     in_b = 2 if wl.dtype == torch.bfloat16 else 4
     ncr, ncc = wl.n_comp_rows, wl.n_comp_cols
-    seed = wl.seed * 1000 + rank
+    seed = ranks.shard_seed(wl.seed, rank)
     stream = torch.cuda.Stream(device=dev)
     n_windows = max(1, wl.decode_tokens // W)
 
@@ -342,7 +330,7 @@ def run_ours(args, rank, world, local):
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_gbs()
     # weak scaling: the job's tokens are every rank's tokens over the slowest rank's time
-    value = world * wl.batch * W * L * K / (ms_total * 1e-3)
+    value = ranks.whole_job_rate(wl.batch * W * L * K, world, ms_total * 1e-3)
 
     # ---- comparators on the same workload (same inputs recipe, same rotation)
     comps = {}
@@ -371,7 +359,7 @@ def run_ours(args, rank, world, local):
             e1.record(stream)
         torch.cuda.synchronize()
         ms = max_over_ranks(e0.elapsed_time(e1), world) / Kc
-        comps[mode] = {"value": world * wl.batch * W * L / (ms * 1e-3), "ms_per_step": ms,
+        comps[mode] = {"value": ranks.whole_job_rate(wl.batch * W * L, world, ms * 1e-3), "ms_per_step": ms,
                        "hbm_gbs": units * nbytes * W * L / (ms * 1e-3) / 1e9,
                        "bytes_per_unit_token": nbytes}
         del g, stk
@@ -415,7 +403,7 @@ def run_ours(args, rank, world, local):
         e1.record(stream)
         torch.cuda.synchronize()
         ms = max_over_ranks(e0.elapsed_time(e1), world) / Ke
-        e2e = {"value": world * wl.batch * W * L / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+        e2e = {"value": ranks.whole_job_rate(wl.batch * W * L, world, ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "path": "DecodeState.decode_step/flush (C ABI), pinned host inputs copied in and outputs copied out each step"}
 
@@ -507,8 +495,7 @@ def main():
         ap.error("--warmup must be >= 3")
 
     if args.impl == "reference":
-        rank = int(os.environ.get("RANK", "0"))
-        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank, world, _ = ranks.env_ranks()
         res = run_reference(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
