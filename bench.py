@@ -86,6 +86,28 @@ def naive_bytes(d: int, in_b: int, kda: bool) -> int:
 
 # --------------------------------------------------------------- environment
 
+def profiled_traffic(workload: str, kernel: str) -> tuple[int | None, str]:
+    """DRAM bytes (read + write) per launch from the committed ncu summary of
+    `kernel` on `workload`, or None when there is none or when a kernel source
+    it names has changed since the capture (its sha256 no longer matches)."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None, "no ncu capture of this workload"
+    srcs = re.findall(r"^kernel-source: (\S+) sha256 ([0-9a-f]{64})$", text, re.M)
+    m = re.search(r"^traffic_bytes_per_launch: (\d+)$", text, re.M)
+    if not srcs or not m:
+        return None, "capture has no traffic figure"
+    for rel, digest in srcs:
+        with open(os.path.join(ROOT, "recurrent_state_quantization_lq_b200", rel), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != digest:
+                return None, f"kernel changed since the capture ({rel})"
+    return int(m.group(1)), f"ncu dram__bytes_read.sum + dram__bytes_write.sum, profiles/{kernel}_{workload}.md"
+
+
 def measured_hbm_gbs() -> tuple[float, str]:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -419,9 +441,11 @@ def run_ours(args, rank, world, local):
                          f"(windowed mode, W={W}, dense FP64 recurrence), {secs:.1f} s"}
 
     clocks = clk.summary()
+    traffic, traffic_src = profiled_traffic(wl.name, "decode_window")
     roofline = {"bound": "hbm", "kernel": "decode_window_kernel", "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} HBM copy (MEASURED_PEAKS.json hbm_gbs)"
-                if peak_kind == "measured" else "fallback 6.65 TB/s", "traffic": None,
+                if peak_kind == "measured" else "fallback 6.65 TB/s", "traffic": traffic,
+                "traffic_source": traffic_src,
                 "frac_of_nominal_8TBs": achieved / NOMINAL_HBM_GBS,
                 "avg_launch_us": dec_avg_us, "bytes_per_launch": dec_bytes / n_dec}
     res = {
@@ -487,7 +511,7 @@ def main():
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--comparator-steps", type=int, default=40)
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--cpu-tokens", type=int, default=192)
+    ap.add_argument("--cpu-tokens", type=int, default=768)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
