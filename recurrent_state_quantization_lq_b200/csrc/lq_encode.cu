@@ -63,30 +63,51 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Warp-wide argmax over `n` scores with ties to the lower index; entries with
-// score < 0 are excluded.  Every lane returns the winner.
-__device__ int warp_argmax(const float *score, int n) {
+// The indices of the `n` (<= 8) largest of the D (<= 128) non-negative
+// scores, in order, ties to the lower index, packed one byte each (0xff when
+// unused); every lane of every calling warp returns the same list.  Non-negative floats order like their bit patterns, so each
+// pick is one integer maximum over the warp and the lowest index holding it
+// (a ballot per 32 scores); taken scores drop out of later picks.
+template <int D>
+__device__ __forceinline__ uint2 select_top(const float *score, int n) {
+    static_assert(D <= 128, "indices are packed in bytes");
+    uint2 sel = make_uint2(0xffffffffu, 0xffffffffu);
     const int lane = threadIdx.x & 31;
-    float best = -1.0f;
-    int bi = 0x7fffffff;
-    for (int i = lane; i < n; i += 32) {
-        const float s = score[i];
-        if (s > best) { best = s; bi = i; }   // i increases: strict '>' keeps the lower index
-    }
+    uint32_t key[D / 32];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+    for (int k = 0; k < D / 32; ++k) key[k] = __float_as_uint(score[k * 32 + lane]);
+    uint32_t taken = 0;                        // bit k: this lane's score k is taken
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        if (c < n) {
+            uint32_t mx = 0;
+#pragma unroll
+            for (int k = 0; k < D / 32; ++k) mx = max(mx, ((taken >> k) & 1u) ? 0u : key[k]);
+            mx = __reduce_max_sync(0xffffffffu, mx);
+            int idx = -1;
+#pragma unroll
+            for (int k = 0; k < D / 32; ++k) {
+                const uint32_t hit = __ballot_sync(0xffffffffu, !((taken >> k) & 1u) && key[k] == mx);
+                if (idx < 0 && hit != 0u) idx = k * 32 + __ffs(hit) - 1;
+            }
+            const uint32_t keep = ~(0xffu << (8 * (c & 3))), put = (uint32_t)idx << (8 * (c & 3));
+            if (c < 4) sel.x = (sel.x & keep) | put;
+            else sel.y = (sel.y & keep) | put;
+            if ((idx & 31) == lane) taken |= 1u << (idx >> 5);
+        }
     }
-    return bi;
+    return sel;
 }
 
-// Codec scratch in shared memory (floats): per-ty column partials, scores,
-// reciprocal smoothing factors, selections.
+__device__ __forceinline__ int sel_at(uint2 sel, int c) {
+    return (int)(((c < 4 ? sel.x : sel.y) >> (8 * (c & 3))) & 0xffu);
+}
+
+// Codec scratch in shared memory (floats): per-warp column partial sums and
+// maxima (8 x D each), column scores, column maxima, reciprocal smoothing factors.
 template <int D>
 struct CodecScratch {
-    static constexpr int PART = 0, SCORE = 16 * D, RS = 17 * D, SEL = 18 * D, FLOATS = 18 * D + 32;
+    static constexpr int PSUM = 0, PMAX = 8 * D, SCORE = 16 * D, CMAX = 17 * D, RS = 18 * D, FLOATS = 19 * D;
 };
 
 template <int D>
@@ -103,14 +124,15 @@ struct Tile {
 // Steps 2-4 of the codec on the tile in registers, plus the stores.  Called by
 // exactly the kTile tile threads (tid < kTile).
 template <int D, bool KDA>
-__device__ void codec_store(Tile<D> &T, int u, const Views &w, int n_rows, int n_cols, int smooth, int select,
-                            float *scratch) {
+__device__ __forceinline__ void codec_store(Tile<D> &T, int u, const Views &w, int n_rows, int n_cols, int smooth,
+                                            int select, float *scratch) {
     using CS = CodecScratch<D>;
     constexpr int G = Tile<D>::G, NR = Tile<D>::NR;
-    float *sh_part = scratch + CS::PART, *sh_score = scratch + CS::SCORE, *sh_rs = scratch + CS::RS;
-    int *sh_sel = reinterpret_cast<int *>(scratch + CS::SEL);
-    const int tid = T.tid, tx = T.tx, ty = T.ty;
+    float *sh_psum = scratch + CS::PSUM, *sh_pmax = scratch + CS::PMAX, *sh_score = scratch + CS::SCORE;
+    float *sh_cmax = scratch + CS::CMAX, *sh_rs = scratch + CS::RS;
+    const int tid = T.tid, tx = T.tx, ty = T.ty, lane = tid & 31;
     const bool l2 = (select == LQ_SELECT_L2);
+    int32_t *cidx = w.comp_index + (size_t)u * w.comp_index_stride;
     tile_sync();   // the scratch of the previous unit is free
 
     // ------------------------------------------------- 2a. compensator rows
@@ -127,99 +149,94 @@ __device__ void codec_store(Tile<D> &T, int u, const Views &w, int n_rows, int n
             if (tx == 0) sh_score[T.row(r)] = p;
         }
         tile_sync();
-        if (tid < 32) {
-            for (int c = 0; c < n_rows; ++c) {
-                const int i = warp_argmax(sh_score, D);
-                if (tid == 0) {
-                    sh_sel[c] = i;
-                    sh_score[i] = -1.0f;
-                    w.comp_index[(size_t)u * w.comp_index_stride + c] = i;
-                }
-                __syncwarp();
-            }
+        const uint2 sel = select_top<D>(sh_score, n_rows);
+        if (tid == 0) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (c < n_rows) cidx[c] = sel_at(sel, c);
         }
-        tile_sync();
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
-            for (int c = 0; c < n_rows; ++c) {
-                if (sh_sel[c] == T.row(r)) {
-                    float *dst = w.comp_row_vec + ((size_t)u * n_rows + c) * D;
+            int slot = -1;
 #pragma unroll
-                    for (int g = 0; g < G; ++g)
-                        *reinterpret_cast<float4 *>(dst + g * 64 + tx * 4) =
-                            make_float4(T.at(r, g * 4), T.at(r, g * 4 + 1), T.at(r, g * 4 + 2), T.at(r, g * 4 + 3));
+            for (int c = 0; c < 8; ++c)
+                if (c < n_rows && sel_at(sel, c) == T.row(r)) slot = c;
+            if (slot >= 0) {
+                float *dst = w.comp_row_vec + ((size_t)u * n_rows + slot) * D;
 #pragma unroll
-                    for (int m = 0; m < NR / 2; ++m) T.acc[r][m] = make_float2(0.0f, 0.0f);
-                }
+                for (int g = 0; g < G; ++g)
+                    *reinterpret_cast<float4 *>(dst + g * 64 + tx * 4) =
+                        make_float4(T.at(r, g * 4), T.at(r, g * 4 + 1), T.at(r, g * 4 + 2), T.at(r, g * 4 + 3));
+#pragma unroll
+                for (int m = 0; m < NR / 2; ++m) T.acc[r][m] = make_float2(0.0f, 0.0f);
             }
         }
     }
 
-    // ---------------------------------------------- 2b. compensator columns
-    if (n_cols > 0) {
-#pragma unroll
-        for (int c = 0; c < NR; ++c) {
-            float p = 0.0f;
-#pragma unroll
-            for (int r = 0; r < NR; ++r) {
-                const float x = fabsf(T.at(r, c));
-                p = l2 ? p + x * x : fmaxf(p, x);
-            }
-            sh_part[ty * D + T.col(c)] = p;
-        }
-        tile_sync();
-        for (int j = tid; j < D; j += kTile) {
-            float p = 0.0f;
-            for (int y = 0; y < 16; ++y) {
-                const float x = sh_part[y * D + j];
-                p = l2 ? p + x : fmaxf(p, x);
-            }
-            sh_score[j] = p;
-        }
-        tile_sync();
-        if (tid < 32) {
-            for (int c = 0; c < n_cols; ++c) {
-                const int j = warp_argmax(sh_score, D);
-                if (tid == 0) {
-                    sh_sel[16 + c] = j;
-                    sh_score[j] = -1.0f;
-                    w.comp_index[(size_t)u * w.comp_index_stride + n_rows + c] = j;
-                }
-                __syncwarp();
-            }
-        }
-        tile_sync();
-#pragma unroll
-        for (int c = 0; c < NR; ++c) {
-            for (int cc = 0; cc < n_cols; ++cc) {
-                if (sh_sel[16 + cc] == T.col(c)) {
-                    float *dst = w.comp_col_vec + ((size_t)u * n_cols + cc) * D;
-#pragma unroll
-                    for (int g = 0; g < G; ++g)
-                        *reinterpret_cast<float4 *>(dst + g * 64 + ty * 4) = make_float4(
-                            T.at(g * 4, c), T.at(g * 4 + 1, c), T.at(g * 4 + 2, c), T.at(g * 4 + 3, c));
-#pragma unroll
-                    for (int r = 0; r < NR; ++r) T.at(r, c) = 0.0f;
-                }
-            }
-        }
-    }
-
-    // ------------------------------------------------------- 3. smoothing
+    // ------------------- 2b, 3. column statistics of the row-zeroed residual
+    // One pass gives each column's score (sum of squares, or max) and its max.
+    // Zeroing the chosen columns leaves the other columns' maxima unchanged
+    // and makes their own zero, so the smoothing factors follow from the same pass.
 #pragma unroll
     for (int c = 0; c < NR; ++c) {
-        float m = 0.0f;
+        float sq = 0.0f, mx = 0.0f;
 #pragma unroll
-        for (int r = 0; r < NR; ++r) m = fmaxf(m, fabsf(T.at(r, c)));
-        sh_part[ty * D + T.col(c)] = m;
+        for (int r = 0; r < NR; ++r) {
+            const float x = fabsf(T.at(r, c));
+            sq = sq + x * x;
+            mx = fmaxf(mx, x);
+        }
+        sq += __shfl_xor_sync(0xffffffffu, sq, 16);          // the warp's two rows of tx groups
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        if (lane < 16) {
+            sh_psum[(ty >> 1) * D + T.col(c)] = sq;
+            sh_pmax[(ty >> 1) * D + T.col(c)] = mx;
+        }
     }
     tile_sync();
     for (int j = tid; j < D; j += kTile) {
-        float m = 0.0f;
-        for (int y = 0; y < 16; ++y) m = fmaxf(m, sh_part[y * D + j]);
+        float sq = 0.0f, mx = 0.0f;
+#pragma unroll
+        for (int y = 0; y < 8; ++y) {
+            sq += sh_psum[y * D + j];
+            mx = fmaxf(mx, sh_pmax[y * D + j]);
+        }
+        sh_score[j] = l2 ? sq : mx;
+        sh_cmax[j] = mx;
+    }
+    tile_sync();
+    const uint2 csel = select_top<D>(sh_score, n_cols);
+    if (tid == 0) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            if (c < n_cols) cidx[n_rows + c] = sel_at(csel, c);
+    }
+    for (int j = tid; j < D; j += kTile) {
+        bool chosen = false;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) chosen |= (c < n_cols && sel_at(csel, c) == j);
+        const float m = chosen ? 0.0f : sh_cmax[j];
         const float s = (smooth && m > 0.0f) ? __fsqrt_rn(m) : 1.0f;
         sh_rs[j] = __fdiv_rn(1.0f, s);          // applied as a multiplication
         if (w.col_smooth != nullptr) w.col_smooth[(size_t)u * D + j] = s;
+    }
+    if (n_cols > 0) {
+#pragma unroll
+        for (int c = 0; c < NR; ++c) {
+            int slot = -1;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc)
+                if (cc < n_cols && sel_at(csel, cc) == T.col(c)) slot = cc;
+            if (slot >= 0) {
+                float *dst = w.comp_col_vec + ((size_t)u * n_cols + slot) * D;
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+                    *reinterpret_cast<float4 *>(dst + g * 64 + ty * 4) =
+                        make_float4(T.at(g * 4, c), T.at(g * 4 + 1, c), T.at(g * 4 + 2, c), T.at(g * 4 + 3, c));
+#pragma unroll
+                for (int r = 0; r < NR; ++r) T.at(r, c) = 0.0f;
+            }
+        }
     }
     tile_sync();
 
@@ -227,27 +244,38 @@ __device__ void codec_store(Tile<D> &T, int u, const Views &w, int n_rows, int n
     float rs[NR];
 #pragma unroll
     for (int c = 0; c < NR; ++c) rs[c] = sh_rs[T.col(c)];
-    int8_t *Qu = w.codes + (size_t)u * D * D;
+    float m[NR];
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
-        float m = 0.0f;
+        float mm = 0.0f;
 #pragma unroll
         for (int c = 0; c < NR; ++c) {
             T.at(r, c) = __fmul_rn(T.at(r, c), rs[c]);
-            m = fmaxf(m, fabsf(T.at(r, c)));
+            mm = fmaxf(mm, fabsf(T.at(r, c)));
         }
-        m = group_max<16>(m);
-        const float sigma = __fdiv_rn(m, 127.0f);
-        const float rho = (m > 0.0f) ? __fdiv_rn(127.0f, m) : 0.0f;
-        if (tx == 0) w.row_scale[(size_t)u * D + T.row(r)] = sigma;
+        m[r] = group_max<16>(mm);
+    }
+    // lane tx divides for row tx mod NR of its group; the rest take rho by shuffle
+    float mine = m[0];
+#pragma unroll
+    for (int r = 1; r < NR; ++r) mine = ((tx & (NR - 1)) == r) ? m[r] : mine;
+    const float rho_mine = (mine > 0.0f) ? __fdiv_rn(127.0f, mine) : 0.0f;
+    if (tx < NR) w.row_scale[(size_t)u * D + T.row(tx)] = __fdiv_rn(mine, 127.0f);
+    int8_t *Qu = w.codes + (size_t)u * D * D;
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        const float rho = __shfl_sync(0xffffffffu, rho_mine, (lane & 16) + r);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            uint32_t word = 0;
+            // rint by adding 1.5 * 2^23 (|x| <= 127.5 here, so the sum is exact
+            // up to the one rounding to an integer, to nearest, ties to even);
+            // the code is then the low byte of the sum's bit pattern.  |x rho|
+            // never exceeds 127 (rho = 127 / max of the row), so no clamp is needed.
+            uint32_t b[4];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float code = fminf(fmaxf(rintf(__fmul_rn(T.at(r, g * 4 + c), rho)), -127.0f), 127.0f);
-                word |= (uint32_t)((int)code & 0xff) << (8 * c);
-            }
+            for (int c = 0; c < 4; ++c)
+                b[c] = __float_as_uint(__fadd_rn(__fmul_rn(T.at(r, g * 4 + c), rho), 12582912.0f));
+            const uint32_t word = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
             *reinterpret_cast<uint32_t *>(Qu + (size_t)T.row(r) * D + g * 64 + tx * 4) = word;
         }
     }
