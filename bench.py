@@ -248,6 +248,8 @@ class LayerStack:
         for l, st in enumerate(self.states):
             st.prefill(prefill_states[l] if prefill_states is not None else None)
         self.T = tokens_per_layer
+        # the states and tokens were made on the current stream; the graphs run on another
+        torch.cuda.synchronize()
 
     def decode(self, l, t):
         tb = self.tok[l]
@@ -473,6 +475,124 @@ def run_ours(args, rank, world, local):
 
 # ------------------------------------------------------------ reference arm
 
+def quality(wl, dev, n_tokens: int | None = None) -> dict:
+    """Windowed INT8, naive per-token INT8 and the FP32 state decode the same
+    inputs from the same start state; the output error of each INT8 mode
+    against the FP32 state, relative L2 per window and overall.
+
+    Tokens are drawn per window on the device (seed = workload seed x 1000 +
+    window index), so the run needs no more than one window of inputs."""
+    from recurrent_state_quantization_lq_b200 import lq
+    B, H, d, W = wl.batch, wl.heads, wl.d_k, wl.window
+    T = n_tokens or wl.decode_tokens
+    gate = "channel" if wl.per_channel_gate else "scalar"
+    seed = wl.seed * 1000
+    if wl.planted:
+        S0 = inputs.planted_state(seed, B, H, d, d)[0].to(dev)
+    elif wl.prefill_tokens:
+        S0 = fp32_prefill(wl, 1, dev, seed)[0]
+    else:
+        S0 = None
+    states = {m: lq.DecodeState(B, H, d, window=W, n_comp_rows=wl.n_comp_rows, n_comp_cols=wl.n_comp_cols,
+                                gate=gate, mode=m, in_dtype=wl.dtype, device=dev)
+              for m in ("window", "naive", "fp32")}
+    for st in states.values():
+        st.prefill(S0)
+    out = {m: torch.empty(B, H, d, dtype=torch.float32, device=dev) for m in states}
+    n_win = (T + W - 1) // W
+    acc = torch.zeros(n_win, 3, dtype=torch.float64, device=dev)   # windowed, naive, reference energy
+    for wi in range(n_win):
+        n = min(W, T - wi * W)
+        tb = inputs.tokens_on_device(seed + wi, n, B, H, d, d, wl.per_channel_gate, wl.dtype, dev)
+        for i in range(n):
+            for m, st in states.items():
+                st.decode_step(tb.q[i], tb.k[i], tb.v[i], tb.g[i], tb.beta[i], out=out[m])
+            ref = out["fp32"].double()
+            acc[wi, 0] += (out["window"].double() - ref).square().sum()
+            acc[wi, 1] += (out["naive"].double() - ref).square().sum()
+            acc[wi, 2] += ref.square().sum()
+        states["window"].flush()
+    for st in states.values():
+        if st.device_status() != lq.LQ_OK:
+            raise RuntimeError(f"device error: {lq.last_error()}")
+    a = acc.cpu()
+    per = (a[:, :2] / a[:, 2:3]).sqrt()
+    tot = (a[:, :2].sum(0) / a[:, 2].sum()).sqrt()
+    return {"rel_l2_windowed_vs_fp32": float(tot[0]), "rel_l2_naive_vs_fp32": float(tot[1]),
+            "naive_over_windowed": float(tot[1] / tot[0]) if tot[0] > 0 else None,
+            "per_window": {"windowed": [float(x) for x in per[:, 0]], "naive": [float(x) for x in per[:, 1]]},
+            "tokens": T, "units": B * H}
+
+
+def sweep(dev, batches=(1, 8, 64, 256, 512), windows=(16, 32, 64, 128, 256), reps: int = 5) -> list[dict]:
+    """Decode throughput of windowed INT8, naive per-token INT8 and the FP32
+    state over a batch x window grid (32 heads, 128 x 128, n_c = 4).  Each
+    point rotates enough layer-states to exceed L2 where the graph size
+    allows (at most 8192 launches per captured window); start states are
+    N(0, 0.3^2) (the state's values do not change the work)."""
+    from recurrent_state_quantization_lq_b200 import lq
+    L2 = 126 * 2 ** 20
+    stream = torch.cuda.Stream(device=dev)
+    rows = []
+    for B in batches:
+        for W in windows:
+            wl = inputs.sweep_workload(B, W)
+            d, units = wl.d_k, B * wl.heads
+            for mode in ("window", "naive", "fp32"):
+                if mode != "window" and W != windows[0]:
+                    continue                      # the comparators do not depend on W
+                per_state = lq.workspace_bytes(lq.make_config(B, wl.heads, d, window=W, n_comp_rows=2,
+                                                              n_comp_cols=2, mode=mode, in_dtype=wl.dtype))
+                L = max(2, min(-(-4 * L2 // per_state), 8192 // W, 256))
+                S0 = [0.3 * torch.randn(B, wl.heads, d, d, device=dev) for _ in range(min(L, 4))]
+                stk = LayerStack(wl, L, mode, dev, wl.seed, W, [S0[l % len(S0)] for l in range(L)])
+                del S0
+                with torch.cuda.stream(stream):
+                    for l in range(L):
+                        stk.decode(l, 0)
+                        stk.states[l].flush()
+                torch.cuda.synchronize()
+                if mode == "window":
+                    gd, gf = stk.capture(0, stream)
+                else:                                   # no flush: one graph of decode launches
+                    gd, gf = torch.cuda.CUDAGraph(), None
+                    with torch.cuda.graph(gd, stream=stream):
+                        for i in range(W):
+                            for l in range(L):
+                                stk.decode(l, i)
+                graphs = [g for g in (gd, gf) if g is not None]
+                with torch.cuda.stream(stream):
+                    for g in graphs:
+                        g.replay()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    for _ in range(reps):
+                        for g in graphs:
+                            g.replay()
+                    e1.record(stream)
+                torch.cuda.synchronize()
+                for st in stk.states:
+                    assert st.device_status(stream) == lq.LQ_OK, lq.last_error()
+                ms = e0.elapsed_time(e1) / reps               # one window for every layer-state
+                if mode == "window":
+                    nb = sum(decode_window_bytes(d, 2, False, 2, 2, n) for n in range(W)) / W + \
+                        flush_bytes(d, 2, False, 2, 2, W) / W
+                elif mode == "naive":
+                    nb = naive_bytes(d, 2, False)
+                else:
+                    nb = fp32_bytes(d, 2, False)
+                rows.append({"batch": B, "window": W if mode == "window" else None, "mode": mode,
+                             "tokens_per_s_per_layer": B * W * L / (ms * 1e-3),
+                             "hbm_gbs": units * nb * W * L / (ms * 1e-3) / 1e9,
+                             "bytes_per_unit_token": nb, "layers_rotated": L,
+                             "l2": "working set > L2" if L * per_state > L2 else "working set fits in L2"})
+                del gd, gf, graphs, stk
+                torch.cuda.synchronize()
+    return rows
+
+
 def run_reference(args, rank, world):
     """The oracle, as it stands, on the host cores: the reference arm."""
     if rank != 0:
@@ -514,9 +634,29 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=768)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quality", nargs="?", const="gdn_outlier_b256_h32_d128_w64", default=None,
+                    metavar="WORKLOAD", help="print the output errors of windowed and naive INT8 against the FP32 "
+                    "state on WORKLOAD (default: the outlier-stress workload) instead of timing")
+    ap.add_argument("--quality-tokens", type=int, default=None)
+    ap.add_argument("--sweep", action="store_true",
+                    help="print one JSON line per point of the batch x window throughput sweep instead of timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+
+    if args.quality is not None:
+        torch.cuda.set_device(0)
+        wl = inputs.WORKLOADS[args.quality]
+        res = quality(wl, torch.device("cuda", 0), args.quality_tokens)
+        print(json.dumps({"mode": "quality", "workload": wl.name, "window": wl.window,
+                          "n_comp": wl.n_comp_rows + wl.n_comp_cols, **res}), flush=True)
+        return
+
+    if args.sweep:
+        torch.cuda.set_device(0)
+        for row in sweep(torch.device("cuda", 0)):
+            print(json.dumps({"mode": "sweep", **row}), flush=True)
+        return
 
     if args.impl == "reference":
         rank, world, _ = ranks.env_ranks()

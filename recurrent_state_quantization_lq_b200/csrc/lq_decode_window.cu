@@ -447,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const bool on = c < ncc;
-                jc[c] = on ? cidx[ncr + c] : 0;
+                jc[c] = on ? (cidx[ncr + c] & (D - 1)) : 0;   // in range whatever the workspace holds
                 vcol[c] = on ? ccol[c * D + tid] : 0.0f;
                 if (c < ncr && cidx[c] == tid) rc = c;
             }

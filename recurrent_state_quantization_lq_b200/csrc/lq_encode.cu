@@ -93,7 +93,7 @@ __device__ __forceinline__ uint2 select_top(const float *score, int n) {
             const uint32_t keep = ~(0xffu << (8 * (c & 3))), put = (uint32_t)idx << (8 * (c & 3));
             if (c < 4) sel.x = (sel.x & keep) | put;
             else sel.y = (sel.y & keep) | put;
-            if ((idx & 31) == lane) taken |= 1u << (idx >> 5);
+            if (idx >= 0 && (idx & 31) == lane) taken |= 1u << (idx >> 5);
         }
     }
     return sel;
