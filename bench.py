@@ -288,6 +288,98 @@ def fp32_prefill(wl, n_layers, device, seed):
     return S
 
 
+def run_e2e(win, wl, dev, L: int, W: int, K: int, args, world: int) -> dict:
+    """The step through the public binding with the inputs in pinned host
+    memory: every step copies each token's q, k, v, g, beta (all layers, one
+    packed buffer per token position) to the device, decodes that token
+    through the L layers (a CUDA graph of the binding's calls per token
+    position; the window's last token also flushes every layer) and copies
+    the token's outputs back.  Copies in, compute and copies out run on three
+    streams over a 4-deep ring of device buffers, so token t's outputs
+    travel while token t + 1 computes and token t + 2 arrives."""
+    R = 4
+    assert W % R == 0 or W < R
+    Ke = max(2, min(K, args.e2e_steps))
+    B, H, d = wl.batch, wl.heads, wl.d_k
+    parts = [(l, name) for l in range(L) for name in ("q", "k", "v", "g", "beta")]
+    src = {(l, n): getattr(win.tok[l], n)[:W] for l, n in parts}
+    sizes = [src[p][0].numel() * src[p].element_size() for p in parts]
+    offs = [0]
+    for z in sizes:
+        offs.append(offs[-1] + (z + 255) // 256 * 256)
+    tok_bytes = offs[-1]
+    host_in = torch.empty(W, tok_bytes, dtype=torch.uint8).pin_memory()
+    for i in range(W):
+        for p, o, z in zip(parts, offs, sizes):
+            host_in[i, o:o + z].copy_(src[p][i].contiguous().view(torch.uint8).reshape(-1).cpu())
+    out_bytes = L * B * H * d * 4
+    host_out = torch.empty(W, out_bytes, dtype=torch.uint8).pin_memory()
+    dev_in = torch.empty(R, tok_bytes, dtype=torch.uint8, device=dev)
+    dev_out = torch.empty(R, L, B, H, d, dtype=torch.float32, device=dev)
+
+    def view(r, p):
+        l, n = p
+        j = parts.index(p)
+        t = src[p]
+        return dev_in[r, offs[j]:offs[j] + sizes[j]].view(t.dtype).view(t.shape[1:])
+
+    s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    graphs = []
+    torch.cuda.synchronize()
+    for i in range(W):
+        r = i % R
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s_comp):
+            for l in range(L):
+                win.states[l].decode_step(view(r, (l, "q")), view(r, (l, "k")), view(r, (l, "v")),
+                                          view(r, (l, "g")), view(r, (l, "beta")), out=dev_out[r, l])
+            if i == W - 1:
+                for st in win.states:
+                    st.flush()
+        graphs.append(g)
+    ev = {k: [torch.cuda.Event() for _ in range(R)] for k in ("in", "comp", "out")}
+
+    def step():
+        for i in range(W):
+            r = i % R
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev["comp"][r])          # the slot's previous inputs are consumed
+                dev_in[r].copy_(host_in[i], non_blocking=True)
+                ev["in"][r].record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev["in"][r])
+                s_comp.wait_event(ev["out"][r])         # the slot's previous outputs are on the host
+                graphs[i].replay()
+                ev["comp"][r].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev["comp"][r])
+                host_out[i].copy_(dev_out[r].view(torch.uint8).reshape(-1), non_blocking=True)
+                ev["out"][r].record(s_out)
+
+    for e in ev.values():
+        for x in e:
+            x.record(s_out)
+    step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    s_comp.wait_event(e0)
+    s_out.wait_event(e0)
+    for _ in range(Ke):
+        step()
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_comp)
+    e1.record(s_out)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / Ke
+    del graphs
+    return {"value": ranks.whole_job_rate(B * W * L, world, ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": W * sum(sizes), "d2h_bytes_per_step": W * out_bytes,
+            "path": "DecodeState.decode_step/flush (C ABI) per token through all layers, in CUDA graphs; "
+                    "pinned host inputs copied in and outputs copied out every token on separate streams"}
+
+
 def run_ours(args, rank, world, local):
     from recurrent_state_quantization_lq_b200 import lq
     dev = torch.device("cuda", local)
@@ -392,44 +484,7 @@ def run_ours(args, rank, world, local):
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        Ke = max(2, min(K, args.e2e_steps))
-        tb0 = [inputs.TokenBatch(*(x[:W].cpu().pin_memory() for x in (tb.q, tb.k, tb.v, tb.g, tb.beta)))
-               for tb in win.tok]
-        dev_in = [inputs.TokenBatch(*(torch.empty_like(x, device=dev) for x in (tb.q, tb.k, tb.v, tb.g, tb.beta)))
-                  for tb in tb0]
-        out_dev = torch.empty(L, W, wl.batch, wl.heads, wl.d_v, dtype=torch.float32, device=dev)
-        out_host = torch.empty(out_dev.shape, dtype=torch.float32).pin_memory()
-        h2d = sum(x.numel() * x.element_size() for tb in tb0 for x in (tb.q, tb.k, tb.v, tb.g, tb.beta))
-        d2h = out_host.numel() * 4
-
-        def e2e_step():
-            with torch.cuda.stream(stream):
-                for l in range(L):
-                    for src, dst in zip((tb0[l].q, tb0[l].k, tb0[l].v, tb0[l].g, tb0[l].beta),
-                                        (dev_in[l].q, dev_in[l].k, dev_in[l].v, dev_in[l].g, dev_in[l].beta)):
-                        dst.copy_(src, non_blocking=True)
-                for i in range(W):
-                    for l in range(L):
-                        b = dev_in[l]
-                        win.states[l].decode_step(b.q[i], b.k[i], b.v[i], b.g[i], b.beta[i], out=out_dev[l, i],
-                                                  stream=stream)
-                for st in win.states:
-                    st.flush(stream=stream)
-                out_host.copy_(out_dev, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        barrier(world)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(Ke):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ms = max_over_ranks(e0.elapsed_time(e1), world) / Ke
-        e2e = {"value": ranks.whole_job_rate(wl.batch * W * L, world, ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "path": "DecodeState.decode_step/flush (C ABI), pinned host inputs copied in and outputs copied out each step"}
+        e2e = run_e2e(win, wl, dev, L, W, K, args, world)
 
     # ---- the oracle on the host cores (rank 0, N = 1 only)
     cpu = None
