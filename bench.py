@@ -530,7 +530,7 @@ def run_ours(args, rank, world, local):
 
 # ------------------------------------------------------------ reference arm
 
-def quality(wl, dev, n_tokens: int | None = None) -> dict:
+def quality(wl, dev, n_tokens: int | None = None, smooth: int = 1) -> dict:
     """Windowed INT8, naive per-token INT8 and the FP32 state decode the same
     inputs from the same start state; the output error of each INT8 mode
     against the FP32 state, relative L2 per window and overall.
@@ -549,7 +549,8 @@ def quality(wl, dev, n_tokens: int | None = None) -> dict:
     else:
         S0 = None
     states = {m: lq.DecodeState(B, H, d, window=W, n_comp_rows=wl.n_comp_rows, n_comp_cols=wl.n_comp_cols,
-                                gate=gate, mode=m, in_dtype=wl.dtype, device=dev)
+                                gate=gate, mode=m, in_dtype=wl.dtype, device=dev,
+                                smooth=smooth if m == "window" else 1)
               for m in ("window", "naive", "fp32")}
     for st in states.values():
         st.prefill(S0)
@@ -648,6 +649,27 @@ def sweep(dev, batches=(1, 8, 64, 256, 512), windows=(16, 32, 64, 128, 256), rep
     return rows
 
 
+def quality_study(dev, tokens: int = 1024) -> list[dict]:
+    """Output error against the FP32 state over window sizes and compensator
+    counts (16 sequences x 32 heads, 128 x 128), on the planted-outlier start
+    state and on a state prefilled by the FP32 recurrence; smoothing off as an
+    ablation at W = 64, n_c = 4."""
+    rows = []
+    points = [(W, nc, 1) for W in (16, 32, 64, 128, 256) for nc in (0, 2, 4, 8)] + [(64, 4, 0)]
+    for planted in (True, False):
+        for W, nc, smooth in points:
+            wl = inputs.Workload(f"gdn_quality_b16_w{W}_nc{nc}", 16, 32, 128, 128, W, nc // 2, nc - nc // 2, False,
+                                 0 if planted else 512, tokens, torch.bfloat16, 3, planted=planted)
+            if not smooth:
+                r = quality(wl, dev, smooth=0)
+            else:
+                r = quality(wl, dev)
+            rows.append({"start": "planted outliers" if planted else "fp32 prefill", "window": W, "n_comp": nc,
+                         "smooth": smooth, "rel_l2_windowed_vs_fp32": r["rel_l2_windowed_vs_fp32"],
+                         "rel_l2_naive_vs_fp32": r["rel_l2_naive_vs_fp32"], "tokens": r["tokens"]})
+    return rows
+
+
 def run_reference(args, rank, world):
     """The oracle, as it stands, on the host cores: the reference arm."""
     if rank != 0:
@@ -693,6 +715,8 @@ def main():
                     metavar="WORKLOAD", help="print the output errors of windowed and naive INT8 against the FP32 "
                     "state on WORKLOAD (default: the outlier-stress workload) instead of timing")
     ap.add_argument("--quality-tokens", type=int, default=None)
+    ap.add_argument("--quality-study", action="store_true",
+                    help="print one JSON line per (start state, W, n_c) point of the output-error study")
     ap.add_argument("--sweep", action="store_true",
                     help="print one JSON line per point of the batch x window throughput sweep instead of timing")
     args = ap.parse_args()
@@ -705,6 +729,12 @@ def main():
         res = quality(wl, torch.device("cuda", 0), args.quality_tokens)
         print(json.dumps({"mode": "quality", "workload": wl.name, "window": wl.window,
                           "n_comp": wl.n_comp_rows + wl.n_comp_cols, **res}), flush=True)
+        return
+
+    if args.quality_study:
+        torch.cuda.set_device(0)
+        for row in quality_study(torch.device("cuda", 0)):
+            print(json.dumps({"mode": "quality_study", **row}), flush=True)
         return
 
     if args.sweep:
