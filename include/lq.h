@@ -41,8 +41,13 @@
  *    device (a gate sum out of the safe range, a bounded wait that expired)
  *    are recorded in the workspace's error word and reported by
  *    lq_device_status().  No kernel traps or asserts.
- *  - Window phase.  All sequences of a handle share one window phase: a
- *    handle counts buffered tokens (lq_window_fill) on the host.
+ *  - Window phase.  By default all sequences of a handle share one window
+ *    phase: the handle counts buffered tokens (lq_window_fill) on the host.
+ *    A ragged handle (cfg.ragged = 1, windowed mode) keeps one count per
+ *    (sequence, head) on the device instead, so that sequences can skip
+ *    steps, join and leave independently (continuous batching); see
+ *    lq_decode_step_active(), lq_window_flush(), lq_window_flush_pending()
+ *    and lq_prefill_sequences().
  *  - Threads.  A handle must not be used by two threads at once.
  */
 #ifndef LQ_H
@@ -83,7 +88,7 @@ enum { LQ_SELECT_L2 = 0, LQ_SELECT_MAXABS = 1 };
 enum { LQ_DTYPE_F32 = 0, LQ_DTYPE_BF16 = 1 };
 
 /* Device error codes in the workspace error word (lq_layout.err, int32[0]). */
-enum { LQ_DEVERR_NONE = 0, LQ_DEVERR_RANGE = 1, LQ_DEVERR_TIMEOUT = 2 };
+enum { LQ_DEVERR_NONE = 0, LQ_DEVERR_RANGE = 1, LQ_DEVERR_TIMEOUT = 2, LQ_DEVERR_WINDOW_FULL = 3 };
 
 typedef struct lq_config {
     int32_t batch;        /* sequences, >= 1                                     */
@@ -98,6 +103,8 @@ typedef struct lq_config {
     int32_t smooth;       /* 1: column smoothing before quantization (windowed)  */
     int32_t select;       /* compensator ranking: LQ_SELECT_L2 or _MAXABS        */
     int32_t in_dtype;     /* dtype of q, k, v: LQ_DTYPE_BF16 or LQ_DTYPE_F32     */
+    int32_t ragged;       /* 1: per-(sequence, head) window phases on the device
+                             (windowed mode only); 0: one shared phase         */
 } lq_config;
 
 /*
@@ -123,6 +130,7 @@ typedef struct lq_layout {
     size_t state_f32;     /* f32   [N][d_v][d_k]                  FP32 mode        */
     int32_t comp_index_stride;  /* n_comp_rows + n_comp_cols rounded up to 4      */
     int32_t window_pad;         /* window rounded up to 4                          */
+    size_t fill;          /* int32 [N] tokens buffered per unit (0..W)   ragged     */
 } lq_layout;
 
 typedef struct lq_state_s *lq_handle;
@@ -163,20 +171,51 @@ LQ_API lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream);
  * corrections, appends (delta_t, key_t, G_t) to the buffer and writes no
  * state; it returns LQ_ERR_WINDOW_FULL when W tokens are already buffered.
  * Naive mode updates and requantizes the INT8 state; FP32 mode updates it.
+ * On a ragged handle this is lq_decode_step_active() with every sequence active.
  */
 LQ_API lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, const void *d_v,
                          const float *d_g, const float *d_beta, float *d_o, void *stream);
+
+/*
+ * Ragged handles: one decode token for every active sequence.  d_active:
+ * device uint8 [batch], nonzero = this sequence takes a token this step; NULL =
+ * all.  Inputs and outputs as lq_decode_step(); the rows of inactive sequences
+ * are not read, their outputs not written and their windows not advanced.  A
+ * unit whose window already holds W tokens is skipped and LQ_DEVERR_WINDOW_FULL
+ * recorded (lq_device_status() returns LQ_ERR_WINDOW_FULL): call
+ * lq_window_flush() after every step.  LQ_ERR_STATE on a shared-phase handle.
+ */
+LQ_API lq_status lq_decode_step_active(lq_handle h, const void *d_q, const void *d_k, const void *d_v,
+                                       const float *d_g, const float *d_beta, const uint8_t *d_active,
+                                       float *d_o, void *stream);
 
 /*
  * End the window (windowed mode; a no-op returning LQ_OK otherwise): rebuild
  * the state in FP32 from the window-start state and the buffered updates,
  * take the new Compensator Tokens (largest rows, then columns), smooth the
  * residual and requantize it to per-row INT8; empty the buffer.  Allowed with
- * any number of buffered tokens, including none.
+ * any number of buffered tokens, including none.  On a ragged handle only the
+ * units whose window holds W tokens are flushed (the others are untouched).
  */
 LQ_API lq_status lq_window_flush(lq_handle h, void *stream);
 
-/* Tokens buffered in the current window (0..W); -1 for a bad handle. */
+/*
+ * Ragged handles: flush every unit holding at least one buffered token (for
+ * example before a sequence leaves).  Shared-phase handles: lq_window_flush().
+ */
+LQ_API lq_status lq_window_flush_pending(lq_handle h, void *stream);
+
+/*
+ * Ragged handles: start new sequences in some batch slots.  The sequences with
+ * d_mask[b] != 0 (device uint8 [batch]) are encoded from d_S0 (device FP32
+ * [batch][heads][d_v][d_k], only their rows read; NULL = all-zero state) and
+ * their windows emptied; the other sequences are untouched.  Requires a prior
+ * lq_prefill_state(); LQ_ERR_STATE on a shared-phase handle.
+ */
+LQ_API lq_status lq_prefill_sequences(lq_handle h, const float *d_S0, const uint8_t *d_mask, void *stream);
+
+/* Tokens buffered in the current window (0..W); -1 for a bad or ragged handle
+ * (a ragged handle's counts are on the device, at lq_layout.fill). */
 LQ_API int32_t lq_window_fill(lq_handle h);
 
 /*

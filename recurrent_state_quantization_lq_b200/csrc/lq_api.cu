@@ -44,6 +44,8 @@ bool validate(const lq_config *c, std::string *why) {
         if (c->smooth != 0 && c->smooth != 1) { *why = "smooth must be 0 or 1"; return false; }
         if (c->select != LQ_SELECT_L2 && c->select != LQ_SELECT_MAXABS) { *why = "select must be LQ_SELECT_L2 or LQ_SELECT_MAXABS"; return false; }
     }
+    if (c->ragged != 0 && c->ragged != 1) { *why = "ragged must be 0 or 1"; return false; }
+    if (c->ragged && c->mode != LQ_MODE_WINDOW) { *why = "ragged window phases need the windowed mode"; return false; }
     return true;
 }
 
@@ -60,7 +62,7 @@ void compute_layout(const lq_config *c, lq_layout *L) {
     lq_layout z;
     z.total_bytes = 0;
     z.err = z.codes = z.row_scale = z.col_smooth = z.comp_index = z.comp_row_vec = z.comp_col_vec = LQ_ABSENT;
-    z.gate_sum = z.buf_delta = z.buf_key = z.buf_gate = z.state_f32 = LQ_ABSENT;
+    z.gate_sum = z.buf_delta = z.buf_key = z.buf_gate = z.state_f32 = z.fill = LQ_ABSENT;
     z.comp_index_stride = 0;
     z.window_pad = 0;
     *L = z;
@@ -86,6 +88,7 @@ void compute_layout(const lq_config *c, lq_layout *L) {
         L->buf_delta = take(N * (size_t)c->window * d * 4);
         L->buf_key = take(N * (size_t)c->window * d * key_b);
         if (c->gate == LQ_GATE_SCALAR) L->buf_gate = take(N * (size_t)L->window_pad * 4);
+        if (c->ragged) L->fill = take(N * 4);
     }
     L->total_bytes = align256(off);
 }
@@ -196,7 +199,10 @@ lq_status lq_state_destroy(lq_handle h) {
     return LQ_OK;
 }
 
-int32_t lq_window_fill(lq_handle h) { return check_handle(h) ? h->n_buf : -1; }
+int32_t lq_window_fill(lq_handle h) {
+    if (!check_handle(h) || h->cfg.ragged) return -1;   // ragged counts live on the device
+    return h->n_buf;
+}
 
 lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream) {
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
@@ -222,17 +228,26 @@ lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream) {
         a.n_cols = win ? c.n_comp_cols : 0;
         a.smooth = win ? c.smooth : 0;
         a.select = win ? c.select : LQ_SELECT_L2;
+        a.fill = nullptr;                  // every unit; the counts are cleared below
+        a.flush_min = 0;
+        a.seq_mask = nullptr;
+        a.heads = c.heads;
         e = lq::launch_encode(a, c.d_k, c.gate, c.in_dtype, s);
         if (e != cudaSuccess) return cuda_fail(e, "launching the encode kernel");
+        if (c.ragged) {
+            e = cudaMemsetAsync(h->ws + h->lay.fill, 0, N * 4, s);
+            if (e != cudaSuccess) return cuda_fail(e, "clearing the window counts");
+        }
     }
     h->n_buf = 0;
     h->prefilled = 1;
     return LQ_OK;
 }
 
-lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, const void *d_v, const float *d_g,
-                         const float *d_beta, float *d_o, void *stream) {
-    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+namespace {
+
+lq_status decode_impl(lq_handle h, const void *d_q, const void *d_k, const void *d_v, const float *d_g,
+                      const float *d_beta, const uint8_t *d_active, float *d_o, void *stream) {
     if (!d_q || !d_k || !d_v || !d_g || !d_beta || !d_o) return fail(LQ_ERR_INVALID_ARG, "NULL input or output");
     if (!aligned(d_q, 16) || !aligned(d_k, 16) || !aligned(d_v, 16))
         return fail(LQ_ERR_INVALID_ARG, "q, k, v must be 16-byte aligned");
@@ -240,7 +255,7 @@ lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, const vo
     if (!aligned(d_g, c.gate == LQ_GATE_CHANNEL ? 16 : 4) || !aligned(d_beta, 4) || !aligned(d_o, 4))
         return fail(LQ_ERR_INVALID_ARG, "g, beta, o misaligned (g per-channel: 16 bytes; others: 4)");
     if (!h->prefilled) return fail(LQ_ERR_STATE, "decode before lq_prefill_state");
-    if (c.mode == LQ_MODE_WINDOW && h->n_buf >= c.window)
+    if (c.mode == LQ_MODE_WINDOW && !c.ragged && h->n_buf >= c.window)
         return fail(LQ_ERR_WINDOW_FULL, "window holds W tokens: call lq_window_flush first");
     if (c.mode == LQ_MODE_WINDOW && !h->codes_map_ready) {
         cudaError_t e = lq::make_codes_map(&h->codes_map, reinterpret_cast<const int8_t *>(h->ws + h->lay.codes),
@@ -253,18 +268,22 @@ lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, const vo
     a.q = d_q; a.k = d_k; a.v = d_v; a.g = d_g; a.beta = d_beta; a.o = d_o;
     a.n_buf = h->n_buf;
     a.codes_map = &h->codes_map;
+    a.fill = c.ragged ? reinterpret_cast<int32_t *>(h->ws + h->lay.fill) : nullptr;
+    a.active = c.ragged ? d_active : nullptr;
+    a.heads = c.heads;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (c.mode == LQ_MODE_WINDOW) e = lq::launch_decode_window(a, c.d_k, c.gate, c.in_dtype, s);
     else if (c.mode == LQ_MODE_NAIVE) e = lq::launch_decode_naive(a, c.d_k, c.gate, c.in_dtype, s);
     else e = lq::launch_decode_fp32(a, c.d_k, c.gate, c.in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "launching the decode kernel");
-    if (c.mode == LQ_MODE_WINDOW) h->n_buf += 1;
+    if (c.mode == LQ_MODE_WINDOW && !c.ragged) h->n_buf += 1;
     return LQ_OK;
 }
 
-lq_status lq_window_flush(lq_handle h, void *stream) {
-    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+// Flush the windowed state: every unit (shared phase), or the units holding at
+// least flush_min buffered tokens (ragged phases).
+lq_status flush_impl(lq_handle h, int flush_min, void *stream) {
     const lq_config &c = h->cfg;
     if (c.mode != LQ_MODE_WINDOW) return LQ_OK;
     if (!h->prefilled) return fail(LQ_ERR_STATE, "flush before lq_prefill_state");
@@ -277,9 +296,63 @@ lq_status lq_window_flush(lq_handle h, void *stream) {
     a.n_cols = c.n_comp_cols;
     a.smooth = c.smooth;
     a.select = c.select;
+    a.fill = c.ragged ? reinterpret_cast<int32_t *>(h->ws + h->lay.fill) : nullptr;
+    a.flush_min = flush_min;
+    a.seq_mask = nullptr;
+    a.heads = c.heads;
     cudaError_t e = lq::launch_encode(a, c.d_k, c.gate, c.in_dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "launching the flush kernel");
     h->n_buf = 0;
+    return LQ_OK;
+}
+
+}  // namespace
+
+lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, const void *d_v, const float *d_g,
+                         const float *d_beta, float *d_o, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    return decode_impl(h, d_q, d_k, d_v, d_g, d_beta, nullptr, d_o, stream);
+}
+
+lq_status lq_decode_step_active(lq_handle h, const void *d_q, const void *d_k, const void *d_v, const float *d_g,
+                                const float *d_beta, const uint8_t *d_active, float *d_o, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    if (!h->cfg.ragged) return fail(LQ_ERR_STATE, "lq_decode_step_active needs a ragged handle");
+    return decode_impl(h, d_q, d_k, d_v, d_g, d_beta, d_active, d_o, stream);
+}
+
+lq_status lq_window_flush(lq_handle h, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    return flush_impl(h, h->cfg.window, stream);
+}
+
+lq_status lq_window_flush_pending(lq_handle h, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    return flush_impl(h, 1, stream);
+}
+
+lq_status lq_prefill_sequences(lq_handle h, const float *d_S0, const uint8_t *d_mask, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    const lq_config &c = h->cfg;
+    if (!c.ragged) return fail(LQ_ERR_STATE, "lq_prefill_sequences needs a ragged handle");
+    if (!h->prefilled) return fail(LQ_ERR_STATE, "lq_prefill_sequences before lq_prefill_state");
+    if (d_mask == nullptr) return fail(LQ_ERR_INVALID_ARG, "NULL sequence mask");
+    if (d_S0 != nullptr && !aligned(d_S0, 16)) return fail(LQ_ERR_INVALID_ARG, "S0 must be 16-byte aligned");
+    lq::EncodeArgs a;
+    a.w = views(h);
+    a.S0 = d_S0;
+    a.from_buffer = 0;
+    a.n_buf = 0;
+    a.n_rows = c.n_comp_rows;
+    a.n_cols = c.n_comp_cols;
+    a.smooth = c.smooth;
+    a.select = c.select;
+    a.fill = reinterpret_cast<int32_t *>(h->ws + h->lay.fill);
+    a.flush_min = 0;
+    a.seq_mask = d_mask;
+    a.heads = c.heads;
+    cudaError_t e = lq::launch_encode(a, c.d_k, c.gate, c.in_dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launching the encode kernel");
     return LQ_OK;
 }
 
@@ -293,6 +366,11 @@ lq_status lq_device_status(lq_handle h, void *stream) {
     if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
     if (word[0] == LQ_DEVERR_NONE) return LQ_OK;
     char buf[160];
+    if (word[0] == LQ_DEVERR_WINDOW_FULL) {
+        snprintf(buf, sizeof buf, "decode into a full window at unit %d (%d tokens buffered): flush after every step",
+                 word[1], word[2]);
+        return fail(LQ_ERR_WINDOW_FULL, buf);
+    }
     if (word[0] == LQ_DEVERR_RANGE) {
         snprintf(buf, sizeof buf, "gate sum outside +-80 at unit %d, key channel %d: flush more often", word[1], word[2]);
         return fail(LQ_ERR_RANGE, buf);

@@ -209,7 +209,7 @@ __device__ __forceinline__ uint32_t digits4(float y, float down) {
     }
     return out;
 }
-template <int D, bool KDA, typename InT, typename KeyT>
+template <int D, bool KDA, typename InT, typename KeyT, bool RAGGED>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_window_kernel(DecodeArgs a, const __grid_constant__ CUtensorMap codes_map) {
     using Sh = Shape<D, KDA, InT, KeyT>;
@@ -217,7 +217,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const Views &w = a.w;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ncr = w.n_comp_rows, ncc = w.n_comp_cols, cis = w.comp_index_stride, ncomp = ncr + ncc;
-    const int n_buf = a.n_buf, nchunks = (n_buf + E - 1) / E, units = w.units;
+    const int units = w.units;
+    // Tokens buffered in unit u's window, and whether it takes a token this step:
+    // one count and every unit active, or (ragged phases) per-unit counts and
+    // per-sequence activity.  The producer and the consumers decide alike.
+    auto unit_fill = [&](int u) -> int { return RAGGED ? a.fill[u] : a.n_buf; };
+    auto unit_active = [&](int u) -> bool { return !RAGGED || a.active == nullptr || a.active[u / a.heads] != 0; };
     const Meta M = meta_layout<D, KDA, InT>(ncr, ncc, cis);
 
     extern __shared__ __align__(1024) unsigned char sm_raw[];
@@ -254,6 +259,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if (++slot == kSlots) { slot = 0; ph ^= 1u; }
         };
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
+            const int n_buf = unit_fill(u);
+            if (!unit_active(u)) continue;
+            if (RAGGED && n_buf >= w.window) {     // ragged phases: the window is full
+                report_error(w.err, LQ_DEVERR_WINDOW_FULL, u, n_buf);
+                continue;
+            }
+            const int nchunks = (n_buf + E - 1) / E;
             unsigned char *dst = acquire(u, -1);
             if (dst == nullptr) return;
             uint64_t *bar = &full[slot];
@@ -316,7 +328,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     int u = blockIdx.x;
     float beta_n = 0.0f, g_n = 0.0f, gam_n = 0.0f;
     double G_n = 0.0;
+    int fill_n = 0;
+    bool active_n = false;
     if (u < units) {
+        fill_n = unit_fill(u);
+        active_n = unit_active(u);
         beta_n = a.beta[u];
         if (!KDA) {
             g_n = a.g[u];
@@ -328,11 +344,23 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const float beta = beta_n;
         const double Gs = G_n;                     // scalar gate: G_t
         const float gam_s = gam_n;                 // scalar gate: gamma_t
+        const int n_buf = fill_n;
+        const bool active = active_n;
         const int un = u + gridDim.x;
         if (un < units) {                          // next unit's scalars, in flight meanwhile
+            fill_n = unit_fill(un);
+            active_n = unit_active(un);
             beta_n = a.beta[un];
             if (!KDA) { g_n = a.g[un]; G_n = w.gate_sum[un]; }
         }
+        if (RAGGED && (!active || n_buf >= w.window)) {   // not decoded this step (nor loaded)
+            if (!KDA && un < units) {
+                G_n = G_n + (double)g_n;
+                gam_n = exp_of_double(G_n);
+            }
+            continue;
+        }
+        const int nchunks = (n_buf + E - 1) / E;
 
         // ------------------------------------------------ A1: operand prep
         bool bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
@@ -598,6 +626,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             w.buf_gate[(size_t)u * w.window_pad + n_buf] = exp_of_double(-Gs);
             w.gate_sum[u] = Gs;
         }
+        if (RAGGED && tid == 0) a.fill[u] = n_buf + 1;
         if (!KDA && un < units) {                  // next unit's G_t and gamma_t, off its critical path
             G_n = G_n + (double)g_n;
             gam_n = exp_of_double(G_n);
@@ -618,12 +647,12 @@ int sm_count() {
     return cached[dev];
 }
 
-template <int D, bool KDA, typename InT, typename KeyT>
-cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
+template <int D, bool KDA, typename InT, typename KeyT, bool RAGGED>
+cudaError_t launch_r(const DecodeArgs &a, cudaStream_t s) {
     using Sh = Shape<D, KDA, InT, KeyT>;
     const Meta M = meta_layout<D, KDA, InT>(a.w.n_comp_rows, a.w.n_comp_cols, a.w.comp_index_stride);
     if (M.bytes > kSlotBytes || D * D > kSlotBytes) return cudaErrorInvalidValue;
-    auto kern = decode_window_kernel<D, KDA, InT, KeyT>;
+    auto kern = decode_window_kernel<D, KDA, InT, KeyT, RAGGED>;
     // The opt-in shared-memory size is set once per device, so that launches
     // inside a stream capture make no attribute calls.
     static bool opted_in[64] = {false};
@@ -638,6 +667,12 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
     const int grid = min(a.w.units, kCtasPerSm * sm_count());
     kern<<<grid, kThreads, Sh::SMEM, s>>>(a, *reinterpret_cast<const CUtensorMap *>(a.codes_map));
     return cudaGetLastError();
+}
+
+// Shared window phases compile without the per-unit counts and the active mask.
+template <int D, bool KDA, typename InT, typename KeyT>
+cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
+    return a.fill != nullptr ? launch_r<D, KDA, InT, KeyT, true>(a, s) : launch_r<D, KDA, InT, KeyT, false>(a, s);
 }
 
 }  // namespace

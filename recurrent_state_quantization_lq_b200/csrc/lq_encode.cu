@@ -298,6 +298,7 @@ __global__ void __launch_bounds__(kTile, 2) prefill_kernel(EncodeArgs a) {
     T.tx = T.tid & 15;
     T.ty = T.tid >> 4;
     const int u = blockIdx.x;
+    if (a.seq_mask != nullptr && a.seq_mask[u / a.heads] == 0) return;   // sequence not restarted
     if (a.S0 != nullptr) {
         const float *S0 = a.S0 + (size_t)u * D * D;
 #pragma unroll
@@ -315,6 +316,7 @@ __global__ void __launch_bounds__(kTile, 2) prefill_kernel(EncodeArgs a) {
             for (int m = 0; m < NR / 2; ++m) T.acc[r][m] = make_float2(0.0f, 0.0f);
     }
     codec_store<D, KDA>(T, u, a.w, a.n_rows, a.n_cols, a.smooth, a.select, pf_scratch);
+    if (a.fill != nullptr && T.tid == 0) a.fill[u] = 0;
 }
 
 // ==================================================================== flush
@@ -354,14 +356,19 @@ __host__ __device__ FlushMeta flush_meta_layout(int ncr, int ncc, int cis) {
     return m;
 }
 
-template <int D, bool KDA, typename KeyT>
+template <int D, bool KDA, typename KeyT, bool RAGGED>
 __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
     using Sh = FlushShape<D, KDA, KeyT>;
     constexpr int G = Tile<D>::G, NR = Tile<D>::NR, E = Sh::E;
     const Views &w = a.w;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ncr = w.n_comp_rows, ncc = w.n_comp_cols, cis = w.comp_index_stride, ncomp = ncr + ncc;
-    const int n_buf = a.n_buf, nchunks = (n_buf + E - 1) / E, units = w.units;
+    const int units = w.units;
+    // Tokens buffered in unit u: one count, or (ragged phases) per-unit counts,
+    // and only units holding at least flush_min tokens are flushed.  The
+    // producer and the tile threads decide alike.
+    auto unit_fill = [&](int u) -> int { return RAGGED ? a.fill[u] : a.n_buf; };
+    auto unit_flushed = [&](int n) -> bool { return !RAGGED || n >= a.flush_min; };
     const FlushMeta M = flush_meta_layout<D, KDA>(ncr, ncc, cis);
 
     extern __shared__ __align__(128) unsigned char sm[];
@@ -398,6 +405,9 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
             if (++slot == kSlots) { slot = 0; ph ^= 1u; }
         };
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
+            const int n_buf = unit_fill(u);
+            if (!unit_flushed(n_buf)) continue;
+            const int nchunks = (n_buf + E - 1) / E;
             unsigned char *dst = acquire(u, -1);
             if (dst == nullptr) return;
             uint64_t *bar = &full[slot];
@@ -451,6 +461,9 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
     for (; u < units; u += gridDim.x) {
         const double GW = G_n;                       // scalar gate: G at the window end
         if (!KDA && u + (int)gridDim.x < units) G_n = w.gate_sum[u + gridDim.x];
+        const int n_buf = unit_fill(u);
+        if (!unit_flushed(n_buf)) continue;
+        const int nchunks = (n_buf + E - 1) / E;
 
         // -------- dequantized window-start state plus compensators (undecayed)
         bool bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
@@ -593,6 +606,7 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
                 for (int m = 0; m < NR / 2; ++m) T.acc[r][m] = __fmul2_rn(T.acc[r][m], gg[m]);
         }
         codec_store<D, KDA>(T, u, w, ncr, ncc, a.smooth, a.select, scratch);
+        if (RAGGED && tid == 0) a.fill[u] = 0;
     }
 }
 
@@ -609,16 +623,12 @@ int sm_count() {
     return cached[dev];
 }
 
-template <int D, bool KDA, typename KeyT>
-cudaError_t launch_encode_t(const EncodeArgs &a, cudaStream_t s) {
-    if (!a.from_buffer) {
-        prefill_kernel<D, KDA><<<a.w.units, kTile, 4 * CodecScratch<D>::FLOATS, s>>>(a);
-        return cudaGetLastError();
-    }
+template <int D, bool KDA, typename KeyT, bool RAGGED>
+cudaError_t launch_flush_r(const EncodeArgs &a, cudaStream_t s) {
     using Sh = FlushShape<D, KDA, KeyT>;
     const FlushMeta M = flush_meta_layout<D, KDA>(a.w.n_comp_rows, a.w.n_comp_cols, a.w.comp_index_stride);
     if (M.bytes > kSlotBytes || D * D > kSlotBytes) return cudaErrorInvalidValue;
-    auto kern = flush_kernel<D, KDA, KeyT>;
+    auto kern = flush_kernel<D, KDA, KeyT, RAGGED>;
     static bool opted_in[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -631,6 +641,16 @@ cudaError_t launch_encode_t(const EncodeArgs &a, cudaStream_t s) {
     const int grid = min(a.w.units, 2 * sm_count());
     kern<<<grid, kFlushThreads, Sh::SMEM, s>>>(a);
     return cudaGetLastError();
+}
+
+// Shared window phases compile without the per-unit counts.
+template <int D, bool KDA, typename KeyT>
+cudaError_t launch_encode_t(const EncodeArgs &a, cudaStream_t s) {
+    if (!a.from_buffer) {
+        prefill_kernel<D, KDA><<<a.w.units, kTile, 4 * CodecScratch<D>::FLOATS, s>>>(a);
+        return cudaGetLastError();
+    }
+    return a.fill != nullptr ? launch_flush_r<D, KDA, KeyT, true>(a, s) : launch_flush_r<D, KDA, KeyT, false>(a, s);
 }
 
 }  // namespace

@@ -17,6 +17,11 @@ struct EncodeArgs {
     int n_cols;        // compensator columns to extract
     int smooth;        // column smoothing on/off
     int select;        // LQ_SELECT_*
+    // ragged window phases: per-unit buffered counts (null: n_buf for every unit)
+    int32_t *fill;
+    int flush_min;     // ragged flush: units holding at least this many tokens
+    const uint8_t *seq_mask;   // prefill: sequences to encode (null: all)
+    int heads;         // units per sequence (for seq_mask)
 };
 
 struct DecodeArgs {
@@ -29,6 +34,11 @@ struct DecodeArgs {
     float *o;
     int n_buf;         // tokens buffered before this one (windowed mode)
     const void *codes_map;   // host copy of the tensor map of the INT8 codes (windowed mode)
+    // ragged window phases: per-unit buffered counts (null: n_buf for every
+    // unit) and per-sequence activity (null: all active)
+    int32_t *fill;
+    const uint8_t *active;
+    int heads;         // units per sequence
 };
 
 // Encode the tensor map the windowed decode uses to load one unit's INT8 tile

@@ -34,14 +34,14 @@ STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED", 3:
 class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "heads", "d_k", "d_v", "window", "n_comp_rows", "n_comp_cols", "gate", "mode",
-        "smooth", "select", "in_dtype")]
+        "smooth", "select", "in_dtype", "ragged")]
 
 
 class Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "total_bytes", "err", "codes", "row_scale", "col_smooth", "comp_index", "comp_row_vec",
         "comp_col_vec", "gate_sum", "buf_delta", "buf_key", "buf_gate", "state_f32")] + \
-        [("comp_index_stride", ctypes.c_int32), ("window_pad", ctypes.c_int32)]
+        [("comp_index_stride", ctypes.c_int32), ("window_pad", ctypes.c_int32), ("fill", ctypes.c_size_t)]
 
 
 class LQError(RuntimeError):
@@ -72,8 +72,14 @@ def lib() -> ctypes.CDLL:
         L.lq_prefill_state.restype = i32
         L.lq_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
         L.lq_decode_step.restype = i32
+        L.lq_decode_step_active.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.lq_decode_step_active.restype = i32
         L.lq_window_flush.argtypes = [vp, vp]
         L.lq_window_flush.restype = i32
+        L.lq_window_flush_pending.argtypes = [vp, vp]
+        L.lq_window_flush_pending.restype = i32
+        L.lq_prefill_sequences.argtypes = [vp, vp, vp, vp]
+        L.lq_prefill_sequences.restype = i32
         L.lq_window_fill.argtypes = [vp]
         L.lq_window_fill.restype = i32
         L.lq_device_status.argtypes = [vp, vp]
@@ -99,9 +105,9 @@ def last_error() -> str:
 
 def make_config(batch: int, heads: int, d: int, window: int = 64, n_comp_rows: int = 2,
                 n_comp_cols: int = 2, gate: str = "scalar", mode: str = "window", smooth: int = 1,
-                select: str = "l2", in_dtype: torch.dtype = torch.bfloat16) -> Config:
+                select: str = "l2", in_dtype: torch.dtype = torch.bfloat16, ragged: bool = False) -> Config:
     return Config(batch, heads, d, d, window, n_comp_rows, n_comp_cols, GATE[gate], MODE[mode],
-                  smooth, SELECT[select], DTYPE[in_dtype])
+                  smooth, SELECT[select], DTYPE[in_dtype], int(ragged))
 
 
 def workspace_bytes(cfg: Config) -> int:
@@ -135,9 +141,11 @@ class DecodeState:
 
     def __init__(self, batch: int, heads: int, d: int, *, window: int = 64, n_comp_rows: int = 2,
                  n_comp_cols: int = 2, gate: str = "scalar", mode: str = "window", smooth: int = 1,
-                 select: str = "l2", in_dtype: torch.dtype = torch.bfloat16, device=None):
+                 select: str = "l2", in_dtype: torch.dtype = torch.bfloat16, ragged: bool = False,
+                 device=None):
         self.cfg = make_config(batch, heads, d, window, n_comp_rows, n_comp_cols, gate, mode, smooth,
-                               select, in_dtype)
+                               select, in_dtype, ragged)
+        self.ragged = bool(ragged)
         dev = torch.device(device) if device is not None else torch.device("cuda")
         if dev.index is None:
             dev = torch.device(dev.type, torch.cuda.current_device())
@@ -168,22 +176,52 @@ class DecodeState:
         self._check(lib().lq_prefill_state(self._h, _ptr(S0), _stream_ptr(stream, self.device)),
                     "lq_prefill_state")
 
-    def decode_step(self, q, k, v, g, beta, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    def decode_step(self, q, k, v, g, beta, out: torch.Tensor | None = None, stream=None,
+                    active: torch.Tensor | None = None) -> torch.Tensor:
+        """One token for every sequence; on a ragged state, for the sequences
+        with active[b] != 0 (uint8 [batch] on the device; None = all)."""
         if out is None:
             out = torch.empty(self.batch, self.heads, self.d, dtype=torch.float32, device=self.device)
         for t, dt in ((q, self.in_dtype), (k, self.in_dtype), (v, self.in_dtype), (g, torch.float32),
                       (beta, torch.float32), (out, torch.float32)):
             assert t.dtype == dt and t.is_contiguous() and t.device == self.device, (t.dtype, t.device)
-        self._check(lib().lq_decode_step(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(out),
-                                         _stream_ptr(stream, self.device)), "lq_decode_step")
+        if active is not None:
+            assert active.dtype == torch.uint8 and active.numel() == self.batch and active.device == self.device
+            self._check(lib().lq_decode_step_active(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                                    _ptr(active), _ptr(out), _stream_ptr(stream, self.device)),
+                        "lq_decode_step_active")
+        else:
+            self._check(lib().lq_decode_step(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(out),
+                                             _stream_ptr(stream, self.device)), "lq_decode_step")
         return out
 
     def flush(self, stream=None) -> None:
+        """End the window (ragged: of every unit whose window is full)."""
         self._check(lib().lq_window_flush(self._h, _stream_ptr(stream, self.device)), "lq_window_flush")
+
+    def flush_pending(self, stream=None) -> None:
+        """Ragged: end the window of every unit holding buffered tokens."""
+        self._check(lib().lq_window_flush_pending(self._h, _stream_ptr(stream, self.device)),
+                    "lq_window_flush_pending")
+
+    def prefill_sequences(self, S0: torch.Tensor | None, mask: torch.Tensor, stream=None) -> None:
+        """Ragged: restart the sequences with mask[b] != 0 (uint8 [batch] on the
+        device) from S0 (FP32 [batch, heads, d, d]; None = zero state)."""
+        if S0 is not None:
+            assert S0.dtype == torch.float32 and S0.is_contiguous() and S0.device == self.device
+            assert S0.numel() == self.batch * self.heads * self.d * self.d
+        assert mask.dtype == torch.uint8 and mask.numel() == self.batch and mask.device == self.device
+        self._check(lib().lq_prefill_sequences(self._h, _ptr(S0), _ptr(mask), _stream_ptr(stream, self.device)),
+                    "lq_prefill_sequences")
 
     @property
     def fill(self) -> int:
+        """Tokens buffered in the shared window; -1 on a ragged state (see fills())."""
         return lib().lq_window_fill(self._h)
+
+    def fills(self) -> torch.Tensor:
+        """Ragged: tokens buffered per (sequence, head), read from the device."""
+        return self.view("fill").clone()
 
     def device_status(self, stream=None) -> int:
         """Synchronize and return the status of the device error word (LQ_OK if clean)."""
@@ -213,6 +251,7 @@ class DecodeState:
             "buf_key": (key_dt, (c.batch, c.heads, c.window, d)),
             "buf_gate": (torch.float32, (c.batch, c.heads, L.window_pad)),
             "state_f32": (torch.float32, (c.batch, c.heads, d, d)),
+            "fill": (torch.int32, (c.batch, c.heads)),
         }[name]
         dt, shape = spec
         n = 1

@@ -12,7 +12,8 @@ def test_exports_every_declared_symbol():
     names = lq.header_symbols()
     assert set(names) >= {"lq_workspace_bytes", "lq_workspace_layout", "lq_state_create",
                           "lq_prefill_state", "lq_decode_step", "lq_window_flush", "lq_window_fill",
-                          "lq_device_status", "lq_state_destroy", "lq_last_error_string"}
+                          "lq_device_status", "lq_state_destroy", "lq_last_error_string",
+                          "lq_decode_step_active", "lq_window_flush_pending", "lq_prefill_sequences"}
     L = lq.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -101,3 +102,39 @@ def test_flush_is_noop_outside_windowed_mode():
                                  ctypes.byref(h)) == lq.LQ_OK
         assert L.lq_window_flush(h, None) == lq.LQ_OK
         L.lq_state_destroy(h)
+
+
+def test_ragged_layout_and_validation():
+    cfg = lq.make_config(3, 5, 128, window=37, ragged=True)
+    L = lq.workspace_layout(cfg)
+    assert L.fill != lq.ABSENT and L.fill % 256 == 0
+    assert L.fill + 15 * 4 <= L.total_bytes
+    shared = lq.workspace_layout(lq.make_config(3, 5, 128, window=37))
+    assert shared.fill == lq.ABSENT
+    for mode in ("naive", "fp32"):
+        assert lq.workspace_bytes(lq.make_config(3, 5, 128, mode=mode, ragged=True)) == 0
+    bad = lq.make_config(3, 5, 128)
+    bad.ragged = 2
+    assert lq.workspace_bytes(bad) == 0
+
+
+def test_ragged_entry_points_check_the_handle_kind():
+    L = lq.lib()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: every call below returns before any launch
+    shared, ragged = ctypes.c_void_p(), ctypes.c_void_p()
+    cs = lq.make_config(2, 3, 64, window=8)
+    cr = lq.make_config(2, 3, 64, window=8, ragged=True)
+    assert L.lq_state_create(ctypes.byref(cs), fake, lq.workspace_bytes(cs), ctypes.byref(shared)) == lq.LQ_OK
+    assert L.lq_state_create(ctypes.byref(cr), fake, lq.workspace_bytes(cr), ctypes.byref(ragged)) == lq.LQ_OK
+    p = ctypes.c_void_p(1 << 21)
+    # shared-phase handles refuse the ragged calls
+    assert L.lq_decode_step_active(shared, p, p, p, p, p, None, p, None) == lq.LQ_ERR_STATE
+    assert L.lq_prefill_sequences(shared, None, p, None) == lq.LQ_ERR_STATE
+    # ragged handles: counts live on the device; order of calls is checked on the host
+    assert L.lq_window_fill(ragged) == -1
+    assert L.lq_window_fill(shared) == 0
+    assert L.lq_prefill_sequences(ragged, None, p, None) == lq.LQ_ERR_STATE      # before lq_prefill_state
+    assert L.lq_window_flush_pending(ragged, None) == lq.LQ_ERR_STATE            # before lq_prefill_state
+    assert L.lq_decode_step_active(ragged, p, p, p, p, p, None, p, None) == lq.LQ_ERR_STATE
+    assert L.lq_state_destroy(shared) == lq.LQ_OK
+    assert L.lq_state_destroy(ragged) == lq.LQ_OK
