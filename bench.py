@@ -234,13 +234,14 @@ class LayerStack:
     """L independent layer-states of one workload, their token inputs and
     CUDA graphs of each window (decode launches, then flushes)."""
 
-    def __init__(self, wl, n_layers, mode, device, seed, tokens_per_layer, prefill_states=None):
+    def __init__(self, wl, n_layers, mode, device, seed, tokens_per_layer, prefill_states=None, ragged=False):
         from recurrent_state_quantization_lq_b200 import lq
         gate = "channel" if wl.per_channel_gate else "scalar"
         self.wl, self.mode, self.L = wl, mode, n_layers
         self.states = [lq.DecodeState(wl.batch, wl.heads, wl.d_k, window=wl.window,
                                       n_comp_rows=wl.n_comp_rows, n_comp_cols=wl.n_comp_cols, gate=gate,
-                                      mode=mode, in_dtype=wl.dtype, device=device) for _ in range(n_layers)]
+                                      mode=mode, in_dtype=wl.dtype, ragged=ragged, device=device)
+                       for _ in range(n_layers)]
         self.tok = [inputs.tokens_on_device(seed * 100 + l, tokens_per_layer, wl.batch, wl.heads, wl.d_k,
                                             wl.d_v, wl.per_channel_gate, wl.dtype, device)
                     for l in range(n_layers)]
@@ -251,9 +252,9 @@ class LayerStack:
         # the states and tokens were made on the current stream; the graphs run on another
         torch.cuda.synchronize()
 
-    def decode(self, l, t):
+    def decode(self, l, t, active=None):
         tb = self.tok[l]
-        self.states[l].decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=self.out[l])
+        self.states[l].decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=self.out[l], active=active)
 
     def capture(self, window_index, stream):
         """Two graphs for one window: W x L decode launches, then L flushes."""
@@ -649,6 +650,88 @@ def sweep(dev, batches=(1, 8, 64, 256, 512), windows=(16, 32, 64, 128, 256), rep
     return rows
 
 
+def ragged_phases(dev, wl, L: int = 4, reps: int = 20) -> list[dict]:
+    """Continuous batching: sequence b of every layer-state starts its window b mod W
+    tokens in, so each step completes the windows of about B / W sequences.  A step
+    is one decode of every sequence and one flush of the full windows, per layer.
+    'serial' runs each layer's flush after its decode on one stream; 'overlap' runs
+    it on a second stream, joined before that layer's next decode, so it overlaps
+    the decodes of the later layers.  Beside them, on the same inputs: 'lockstep'
+    (a shared-phase handle, one flush per window) and 'aligned' (a ragged handle
+    used without masks, so all sequences stay in one phase, flushed every step)."""
+    from recurrent_state_quantization_lq_b200 import lq
+    W, B, d = wl.window, wl.batch, wl.d_k
+    in_b = 2 if wl.dtype == torch.bfloat16 else 4
+    ncr, ncc, kda = wl.n_comp_rows, wl.n_comp_cols, wl.per_channel_gate
+    units = B * wl.heads
+    stream, side = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    S0 = [0.3 * torch.randn(B, wl.heads, d, d, device=dev) for _ in range(L)]
+    nb = sum(decode_window_bytes(d, in_b, kda, ncr, ncc, n) for n in range(W)) + flush_bytes(d, in_b, kda, ncr, ncc, W)
+    rows = []
+    for variant in ("lockstep", "aligned", "serial", "overlap"):
+        rag = variant != "lockstep"
+        stagger = variant in ("serial", "overlap")
+        stk = LayerStack(wl, L, "window", dev, wl.seed, 2 * W, S0, ragged=rag)
+        offset = torch.arange(B, device=dev) % W
+        with torch.cuda.stream(stream):
+            for l in range(L):                  # warm launches outside capture (kernel attributes)
+                stk.decode(l, 0, active=torch.ones(B, dtype=torch.uint8, device=dev) if rag else None)
+                stk.states[l].flush()
+                if rag:
+                    stk.states[l].flush_pending()
+            if stagger:                         # sequence b holds b mod W tokens
+                for i in range(W - 1):
+                    act = (offset > i).to(torch.uint8)
+                    for l in range(L):
+                        stk.decode(l, W + i, active=act)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        evs = [torch.cuda.Event() for _ in range(L)]
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(W):
+                for l in range(L):
+                    if variant == "overlap" and i > 0:
+                        stream.wait_event(evs[l])
+                    stk.decode(l, i)
+                    if variant in ("serial", "aligned"):
+                        stk.states[l].flush()
+                    elif variant == "overlap":
+                        side.wait_stream(stream)
+                        with torch.cuda.stream(side):
+                            stk.states[l].flush()
+                            evs[l].record(side)
+            if variant == "lockstep":
+                for st in stk.states:
+                    st.flush()
+            elif variant == "overlap":
+                stream.wait_stream(side)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        for st in stk.states:
+            assert st.device_status(stream) == lq.LQ_OK, lq.last_error()
+        if rag:
+            fills = torch.stack([st.fills() for st in stk.states]).view(L, B, wl.heads)
+            want = offset if stagger else torch.zeros_like(offset)
+            assert bool((fills == want.view(1, B, 1)).all()), "phases drifted"
+        ms = e0.elapsed_time(e1) / reps                   # W tokens of every sequence, every layer
+        rows.append({"variant": variant, "workload": wl.name, "batch": B, "window": W, "layers_rotated": L,
+                     "tokens_per_s_per_layer": B * W * L / (ms * 1e-3), "ms_per_window": ms,
+                     "hbm_gbs": units * nb * L / (ms * 1e-3) / 1e9,
+                     "launches_per_window": L * (W + (W if stagger else 1))})
+        del g, stk
+        torch.cuda.synchronize()
+    return rows
+
+
 def quality_study(dev, tokens: int = 1024) -> list[dict]:
     """Output error against the FP32 state over window sizes and compensator
     counts (16 sequences x 32 heads, 128 x 128), on the planted-outlier start
@@ -717,6 +800,8 @@ def main():
     ap.add_argument("--quality-tokens", type=int, default=None)
     ap.add_argument("--quality-study", action="store_true",
                     help="print one JSON line per (start state, W, n_c) point of the output-error study")
+    ap.add_argument("--ragged", nargs="?", const="gdn_b64_h32_d128_w64", default=None, metavar="WORKLOAD",
+                    help="print one JSON line per variant of the staggered-phase (continuous batching) timing")
     ap.add_argument("--sweep", action="store_true",
                     help="print one JSON line per point of the batch x window throughput sweep instead of timing")
     args = ap.parse_args()
@@ -735,6 +820,12 @@ def main():
         torch.cuda.set_device(0)
         for row in quality_study(torch.device("cuda", 0)):
             print(json.dumps({"mode": "quality_study", **row}), flush=True)
+        return
+
+    if args.ragged is not None:
+        torch.cuda.set_device(0)
+        for row in ragged_phases(torch.device("cuda", 0), inputs.WORKLOADS[args.ragged], args.layers):
+            print(json.dumps({"mode": "ragged", **row}), flush=True)
         return
 
     if args.sweep:

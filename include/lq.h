@@ -196,6 +196,12 @@ LQ_API lq_status lq_decode_step_active(lq_handle h, const void *d_q, const void 
  * residual and requantize it to per-row INT8; empty the buffer.  Allowed with
  * any number of buffered tokens, including none.  On a ragged handle only the
  * units whose window holds W tokens are flushed (the others are untouched).
+ * Cost on a ragged handle: until an active mask or lq_prefill_sequences() is
+ * used (counting from lq_prefill_state() or lq_window_flush_pending()), every
+ * unit is in the same phase, which the handle follows on the host: the call
+ * launches nothing when no window is full and otherwise flushes like a
+ * shared-phase handle.  Once phases differ, a launch reads every unit's count
+ * and re-encodes only the due units.
  */
 LQ_API lq_status lq_window_flush(lq_handle h, void *stream);
 

@@ -113,6 +113,9 @@ struct lq_state_s {
     int32_t n_buf;
     int prefilled;
     int codes_map_ready;
+    // ragged handles: every unit is known to be in the same window phase
+    // (n_buf tokens) until an active mask or a sequence restart is used
+    int aligned;
 };
 
 namespace {
@@ -187,6 +190,7 @@ lq_status lq_state_create(const lq_config *cfg, void *d_workspace, size_t bytes,
     h->ws = static_cast<unsigned char *>(d_workspace);
     h->n_buf = 0;
     h->prefilled = 0;
+    h->aligned = 0;
     h->codes_map_ready = 0;
     *out = h;
     return LQ_OK;
@@ -241,6 +245,7 @@ lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream) {
     }
     h->n_buf = 0;
     h->prefilled = 1;
+    h->aligned = 1;
     return LQ_OK;
 }
 
@@ -278,6 +283,10 @@ lq_status decode_impl(lq_handle h, const void *d_q, const void *d_k, const void 
     else e = lq::launch_decode_fp32(a, c.d_k, c.gate, c.in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "launching the decode kernel");
     if (c.mode == LQ_MODE_WINDOW && !c.ragged) h->n_buf += 1;
+    if (c.ragged) {
+        if (d_active != nullptr) h->aligned = 0;
+        else if (h->n_buf < c.window) h->n_buf += 1;   // a full window refuses the token on the device
+    }
     return LQ_OK;
 }
 
@@ -287,6 +296,11 @@ lq_status flush_impl(lq_handle h, int flush_min, void *stream) {
     const lq_config &c = h->cfg;
     if (c.mode != LQ_MODE_WINDOW) return LQ_OK;
     if (!h->prefilled) return fail(LQ_ERR_STATE, "flush before lq_prefill_state");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // A ragged handle whose units share one phase flushes like a shared-phase
+    // handle (every unit, or none when none is due) and clears the counts.
+    const bool per_unit = c.ragged && !h->aligned;
+    if (c.ragged && h->aligned && h->n_buf < flush_min) return LQ_OK;
     lq::EncodeArgs a;
     a.w = views(h);
     a.S0 = nullptr;
@@ -296,12 +310,17 @@ lq_status flush_impl(lq_handle h, int flush_min, void *stream) {
     a.n_cols = c.n_comp_cols;
     a.smooth = c.smooth;
     a.select = c.select;
-    a.fill = c.ragged ? reinterpret_cast<int32_t *>(h->ws + h->lay.fill) : nullptr;
+    a.fill = per_unit ? reinterpret_cast<int32_t *>(h->ws + h->lay.fill) : nullptr;
     a.flush_min = flush_min;
     a.seq_mask = nullptr;
     a.heads = c.heads;
-    cudaError_t e = lq::launch_encode(a, c.d_k, c.gate, c.in_dtype, static_cast<cudaStream_t>(stream));
+    cudaError_t e = lq::launch_encode(a, c.d_k, c.gate, c.in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "launching the flush kernel");
+    if (c.ragged && h->aligned) {
+        e = cudaMemsetAsync(h->ws + h->lay.fill, 0, (size_t)c.batch * c.heads * 4, s);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the window counts");
+    }
+    if (c.ragged && flush_min <= 1) h->aligned = 1;     // every unit's window is empty again
     h->n_buf = 0;
     return LQ_OK;
 }
@@ -353,6 +372,7 @@ lq_status lq_prefill_sequences(lq_handle h, const float *d_S0, const uint8_t *d_
     a.heads = c.heads;
     cudaError_t e = lq::launch_encode(a, c.d_k, c.gate, c.in_dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "launching the encode kernel");
+    h->aligned = 0;                       // the restarted sequences start a new phase
     return LQ_OK;
 }
 

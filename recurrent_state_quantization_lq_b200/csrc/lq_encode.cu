@@ -29,6 +29,7 @@
 // shared-memory slots with 1-D bulk async copies and bounded mbarrier waits;
 // eight consumer warps rebuild, encode and store.
 #include "lq_kernels.h"
+#include "lq_select.cuh"
 
 namespace lq {
 namespace {
@@ -61,46 +62,6 @@ __device__ __forceinline__ bool tile_sync_or(bool pred) {
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// The indices of the `n` (<= 8) largest of the D (<= 128) non-negative
-// scores, in order, ties to the lower index, packed one byte each (0xff when
-// unused); every lane of every calling warp returns the same list.  Non-negative floats order like their bit patterns, so each
-// pick is one integer maximum over the warp and the lowest index holding it
-// (a ballot per 32 scores); taken scores drop out of later picks.
-template <int D>
-__device__ __forceinline__ uint2 select_top(const float *score, int n) {
-    static_assert(D <= 128, "indices are packed in bytes");
-    uint2 sel = make_uint2(0xffffffffu, 0xffffffffu);
-    const int lane = threadIdx.x & 31;
-    uint32_t key[D / 32];
-#pragma unroll
-    for (int k = 0; k < D / 32; ++k) key[k] = __float_as_uint(score[k * 32 + lane]);
-    uint32_t taken = 0;                        // bit k: this lane's score k is taken
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        if (c < n) {
-            uint32_t mx = 0;
-#pragma unroll
-            for (int k = 0; k < D / 32; ++k) mx = max(mx, ((taken >> k) & 1u) ? 0u : key[k]);
-            mx = __reduce_max_sync(0xffffffffu, mx);
-            int idx = -1;
-#pragma unroll
-            for (int k = 0; k < D / 32; ++k) {
-                const uint32_t hit = __ballot_sync(0xffffffffu, !((taken >> k) & 1u) && key[k] == mx);
-                if (idx < 0 && hit != 0u) idx = k * 32 + __ffs(hit) - 1;
-            }
-            const uint32_t keep = ~(0xffu << (8 * (c & 3))), put = (uint32_t)idx << (8 * (c & 3));
-            if (c < 4) sel.x = (sel.x & keep) | put;
-            else sel.y = (sel.y & keep) | put;
-            if (idx >= 0 && (idx & 31) == lane) taken |= 1u << (idx >> 5);
-        }
-    }
-    return sel;
-}
-
-__device__ __forceinline__ int sel_at(uint2 sel, int c) {
-    return (int)(((c < 4 ? sel.x : sel.y) >> (8 * (c & 3))) & 0xffu);
 }
 
 // Codec scratch in shared memory (floats): per-warp column partial sums and
@@ -356,19 +317,15 @@ __host__ __device__ FlushMeta flush_meta_layout(int ncr, int ncc, int cis) {
     return m;
 }
 
-template <int D, bool KDA, typename KeyT, bool RAGGED>
+template <int D, bool KDA, typename KeyT>
 __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
     using Sh = FlushShape<D, KDA, KeyT>;
     constexpr int G = Tile<D>::G, NR = Tile<D>::NR, E = Sh::E;
     const Views &w = a.w;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ncr = w.n_comp_rows, ncc = w.n_comp_cols, cis = w.comp_index_stride, ncomp = ncr + ncc;
-    const int units = w.units;
-    // Tokens buffered in unit u: one count, or (ragged phases) per-unit counts,
-    // and only units holding at least flush_min tokens are flushed.  The
-    // producer and the tile threads decide alike.
-    auto unit_fill = [&](int u) -> int { return RAGGED ? a.fill[u] : a.n_buf; };
-    auto unit_flushed = [&](int n) -> bool { return !RAGGED || n >= a.flush_min; };
+    const int units = w.units, n_buf = a.n_buf;      // one window phase for every unit
+    const int nchunks = (n_buf + E - 1) / E;
     const FlushMeta M = flush_meta_layout<D, KDA>(ncr, ncc, cis);
 
     extern __shared__ __align__(128) unsigned char sm[];
@@ -405,9 +362,6 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
             if (++slot == kSlots) { slot = 0; ph ^= 1u; }
         };
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
-            const int n_buf = unit_fill(u);
-            if (!unit_flushed(n_buf)) continue;
-            const int nchunks = (n_buf + E - 1) / E;
             unsigned char *dst = acquire(u, -1);
             if (dst == nullptr) return;
             uint64_t *bar = &full[slot];
@@ -461,9 +415,6 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
     for (; u < units; u += gridDim.x) {
         const double GW = G_n;                       // scalar gate: G at the window end
         if (!KDA && u + (int)gridDim.x < units) G_n = w.gate_sum[u + gridDim.x];
-        const int n_buf = unit_fill(u);
-        if (!unit_flushed(n_buf)) continue;
-        const int nchunks = (n_buf + E - 1) / E;
 
         // -------- dequantized window-start state plus compensators (undecayed)
         bool bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
@@ -606,7 +557,6 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
                 for (int m = 0; m < NR / 2; ++m) T.acc[r][m] = __fmul2_rn(T.acc[r][m], gg[m]);
         }
         codec_store<D, KDA>(T, u, w, ncr, ncc, a.smooth, a.select, scratch);
-        if (RAGGED && tid == 0) a.fill[u] = 0;
     }
 }
 
@@ -623,12 +573,12 @@ int sm_count() {
     return cached[dev];
 }
 
-template <int D, bool KDA, typename KeyT, bool RAGGED>
-cudaError_t launch_flush_r(const EncodeArgs &a, cudaStream_t s) {
+template <int D, bool KDA, typename KeyT>
+cudaError_t launch_flush_t(const EncodeArgs &a, cudaStream_t s) {
     using Sh = FlushShape<D, KDA, KeyT>;
     const FlushMeta M = flush_meta_layout<D, KDA>(a.w.n_comp_rows, a.w.n_comp_cols, a.w.comp_index_stride);
     if (M.bytes > kSlotBytes || D * D > kSlotBytes) return cudaErrorInvalidValue;
-    auto kern = flush_kernel<D, KDA, KeyT, RAGGED>;
+    auto kern = flush_kernel<D, KDA, KeyT>;
     static bool opted_in[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -643,19 +593,21 @@ cudaError_t launch_flush_r(const EncodeArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-// Shared window phases compile without the per-unit counts.
 template <int D, bool KDA, typename KeyT>
 cudaError_t launch_encode_t(const EncodeArgs &a, cudaStream_t s) {
     if (!a.from_buffer) {
         prefill_kernel<D, KDA><<<a.w.units, kTile, 4 * CodecScratch<D>::FLOATS, s>>>(a);
         return cudaGetLastError();
     }
-    return a.fill != nullptr ? launch_flush_r<D, KDA, KeyT, true>(a, s) : launch_flush_r<D, KDA, KeyT, false>(a, s);
+    return launch_flush_t<D, KDA, KeyT>(a, s);
 }
 
 }  // namespace
 
 cudaError_t launch_encode(const EncodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s) {
+    // Shared window phases flush every unit here; ragged phases flush the
+    // units that are due, one thread-block cluster per unit.
+    if (a.from_buffer && a.fill != nullptr) return launch_flush_split(a, d, gate, in_dtype, s);
     const bool kda = (gate == LQ_GATE_CHANNEL);
     const bool bf = (in_dtype == LQ_DTYPE_BF16);
     if (d == 128) {

@@ -47,6 +47,7 @@ cudaError_t make_codes_map(void *map_out, const int8_t *codes, int d, int units)
 
 // d = d_k = d_v in {64, 128}; gate: LQ_GATE_*; in_dtype: LQ_DTYPE_*.
 cudaError_t launch_encode(const EncodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
+cudaError_t launch_flush_split(const EncodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
 cudaError_t launch_decode_window(const DecodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
 cudaError_t launch_decode_fp32(const DecodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
 cudaError_t launch_decode_naive(const DecodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);

@@ -20,19 +20,23 @@ pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda", 0)
 
 
-def _ragged_case(d, gate, dtype, W, nr, nc, B, H, T, seed, join_at=None, p_active=0.7):
+def _ragged_case(d, gate, dtype, W, nr, nc, B, H, T, seed, join_at=None, p_active=0.7, sample=None,
+                 zero_start=False):
     per_channel = gate == "channel"
     tb = inputs.tokens(seed, 0, T, B, H, d, d, per_channel, dtype)
     rng = np.random.default_rng(seed)
     active = rng.random((T, B)) < p_active
-    gen = torch.Generator().manual_seed(seed)
-    S0 = 0.5 * torch.randn(B, H, d, d, generator=gen)
-    S1 = 0.5 * torch.randn(B, H, d, d, generator=gen)          # the state a joining sequence starts from
+    if zero_start:
+        S0 = S1 = None
+    else:
+        gen = torch.Generator().manual_seed(seed)
+        S0 = 0.5 * torch.randn(B, H, d, d, generator=gen)
+        S1 = 0.5 * torch.randn(B, H, d, d, generator=gen)      # the state a joining sequence starts from
     join_seq = 1 % B
 
     st = lq.DecodeState(B, H, d, window=W, n_comp_rows=nr, n_comp_cols=nc, gate=gate, in_dtype=dtype,
                         ragged=True, device=DEV)
-    st.prefill(S0.to(DEV).contiguous())
+    st.prefill(None if zero_start else S0.to(DEV).contiguous())
     tbd = to_device(tb, DEV)
     out = torch.full((T, B, H, d), float("nan"), device=DEV)
     mask = torch.zeros(B, dtype=torch.uint8, device=DEV)
@@ -46,29 +50,34 @@ def _ragged_case(d, gate, dtype, W, nr, nc, B, H, T, seed, join_at=None, p_activ
     assert st.device_status() == lq.LQ_OK, lq.last_error()
     fills = st.fills().cpu().numpy()
     o_gpu = out.cpu().numpy()
+    # every unit's count: its tokens since it last held W (or since its restart)
+    expect = np.zeros(B, dtype=np.int64)
+    for t in range(T):
+        if join_at is not None and t == join_at:
+            expect[join_seq] = 0
+        expect = np.where(active[t], (expect + 1) % W, expect)
+    assert (fills == expect[:, None]).all()
 
     p = oracle_params(d, W, nr, nc, gate, "window")
-    q, k, v, g, beta = unit_inputs(tb, range(B * H))
+    pairs = [(b, h) for b in range(B) for h in range(H)] if sample is None else sample
+    q, k, v, g, beta = unit_inputs(tb, [b * H + h for b, h in pairs])
     got, ref = [], []
-    for b in range(B):
-        for h in range(H):
-            u = b * H + h
-            steps = np.nonzero(active[:, b])[0]
-            segments = [(S0[b, h], steps)]
-            if join_at is not None and b == join_seq:
-                segments = [(S0[b, h], steps[steps < join_at]), (S1[b, h], steps[steps >= join_at])]
-            for S_start, seg in segments:
-                if len(seg) == 0:
-                    continue
-                r = oracle.run(p, S_start.double().numpy()[None], q[u:u + 1, seg], k[u:u + 1, seg],
-                               v[u:u + 1, seg], g[u:u + 1, seg], beta[u:u + 1, seg], snapshots=False)
-                ref.append(r.o[0])
-                got.append(o_gpu[seg, b, h])
-            last = segments[-1][1]
-            assert fills[b, h] == len(last) % W, (b, h, fills[b, h], len(last))
-            # inactive steps leave the output rows untouched
-            idle = np.setdiff1d(np.arange(T), steps)
-            assert np.isnan(o_gpu[idle, b, h]).all()
+    for u, (b, h) in enumerate(pairs):
+        steps = np.nonzero(active[:, b])[0]
+        start = np.zeros((d, d)) if zero_start else S0[b, h].double().numpy()
+        segments = [(start, steps)]
+        if join_at is not None and b == join_seq:
+            segments = [(start, steps[steps < join_at]), (S1[b, h].double().numpy(), steps[steps >= join_at])]
+        for S_start, seg in segments:
+            if len(seg) == 0:
+                continue
+            r = oracle.run(p, S_start[None], q[u:u + 1, seg], k[u:u + 1, seg], v[u:u + 1, seg], g[u:u + 1, seg],
+                           beta[u:u + 1, seg], snapshots=False)
+            ref.append(r.o[0])
+            got.append(o_gpu[seg, b, h])
+        # inactive steps leave the output rows untouched
+        idle = np.setdiff1d(np.arange(T), steps)
+        assert np.isnan(o_gpu[idle, b, h]).all()
     err = rel_l2(np.concatenate(got), np.concatenate(ref))
     assert err <= 1e-3, err
     st.flush_pending()
@@ -78,9 +87,26 @@ def _ragged_case(d, gate, dtype, W, nr, nc, B, H, T, seed, join_at=None, p_activ
 
 
 @pytest.mark.parametrize("d,gate,dtype", [(64, "scalar", torch.bfloat16), (128, "scalar", torch.bfloat16),
-                                          (128, "channel", torch.bfloat16), (64, "scalar", torch.float32)])
+                                          (128, "channel", torch.bfloat16), (64, "scalar", torch.float32),
+                                          (64, "channel", torch.bfloat16), (128, "scalar", torch.float32)])
 def test_ragged_phases_match_per_sequence_oracle(d, gate, dtype):
     _ragged_case(d, gate, dtype, W=8, nr=2, nc=2, B=3, H=2, T=40, seed=31)
+
+
+def test_ragged_max_select_and_no_compensators():
+    _ragged_case(128, "scalar", torch.bfloat16, W=5, nr=0, nc=0, B=2, H=3, T=17, seed=12)
+    _ragged_case(128, "scalar", torch.bfloat16, W=40, nr=8, nc=8, B=2, H=2, T=90, seed=13, p_active=0.9)
+
+
+def test_ragged_many_units_scan_in_passes():
+    """65,536 units: each persistent cluster scans its candidates in more than
+    one pass of 128; the oracle checks a sample of units."""
+    B, H = 2048, 32
+    rng = np.random.default_rng(5)
+    sample = [(int(b), int(h)) for b, h in zip(rng.integers(0, B, 48), rng.integers(0, H, 48))]
+    sample += [(0, 0), (B - 1, H - 1), (B // 2, 7)]
+    _ragged_case(64, "scalar", torch.bfloat16, W=4, nr=1, nc=1, B=B, H=H, T=9, seed=17, sample=sample,
+                 zero_start=True)
 
 
 def test_ragged_join_restarts_one_sequence():
@@ -100,3 +126,80 @@ def test_ragged_decode_into_full_window_is_reported():
     assert (st.fills() == 0).all()
     st.prefill(None)                            # prefill clears the error word
     assert st.device_status() == lq.LQ_OK
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_ragged_without_masks_matches_shared_phase(gate):
+    """No active mask: every unit keeps the same phase, and a ragged handle
+    flushed after every step gives exactly the shared-phase handle's outputs
+    and encoded state."""
+    d, B, H, W, T = 128, 3, 2, 8, 21
+    tb = to_device(inputs.tokens(41, 0, T, B, H, d, d, gate == "channel"), DEV)
+    S0 = (0.5 * torch.randn(B, H, d, d, generator=torch.Generator().manual_seed(41))).to(DEV)
+    rag = lq.DecodeState(B, H, d, window=W, gate=gate, ragged=True, device=DEV)
+    ref = lq.DecodeState(B, H, d, window=W, gate=gate, device=DEV)
+    rag.prefill(S0)
+    ref.prefill(S0)
+    o_rag = torch.empty(T, B, H, d, device=DEV)
+    o_ref = torch.empty(T, B, H, d, device=DEV)
+    for t in range(T):
+        rag.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=o_rag[t])
+        rag.flush()
+        ref.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=o_ref[t])
+        if ref.fill == W:
+            ref.flush()
+    assert rag.device_status() == lq.LQ_OK and ref.device_status() == lq.LQ_OK
+    assert torch.equal(o_rag, o_ref)
+    for name in ("codes", "row_scale", "col_smooth", "comp_index", "buf_delta"):
+        assert torch.equal(rag.view(name), ref.view(name)), name
+    assert (rag.fills() == T % W).all()
+
+
+def test_ragged_phases_realign_after_flush_pending():
+    """Masked steps, then a pending flush (every partial window encoded), then
+    unmasked steps: each unit follows the oracle run over its own tokens, its
+    partial window ending at the pending flush."""
+    d, B, H, W, T1, T2 = 64, 4, 2, 6, 13, 11
+    T = T1 + T2
+    tb = inputs.tokens(23, 0, T, B, H, d, d, False)
+    rng = np.random.default_rng(23)
+    active = np.ones((T, B), dtype=bool)
+    active[:T1] = rng.random((T1, B)) < 0.6
+    S0 = 0.5 * torch.randn(B, H, d, d, generator=torch.Generator().manual_seed(23))
+    st = lq.DecodeState(B, H, d, window=W, n_comp_rows=1, n_comp_cols=1, ragged=True, device=DEV)
+    st.prefill(S0.to(DEV))
+    tbd = to_device(tb, DEV)
+    out = torch.full((T, B, H, d), float("nan"), device=DEV)
+    for t in range(T):
+        if t == T1:
+            st.flush_pending()
+        if t < T1:
+            act = torch.tensor(active[t].astype(np.uint8), device=DEV)
+            st.decode_step(tbd.q[t], tbd.k[t], tbd.v[t], tbd.g[t], tbd.beta[t], out=out[t], active=act)
+        else:
+            st.decode_step(tbd.q[t], tbd.k[t], tbd.v[t], tbd.g[t], tbd.beta[t], out=out[t])
+        st.flush()
+    assert st.device_status() == lq.LQ_OK, lq.last_error()
+    assert (st.fills() == T2 % W).all()
+    o_gpu = out.cpu().numpy()
+    p = oracle_params(d, W, 1, 1, "scalar", "window")
+    q, k, v, g, beta = unit_inputs(tb, range(B * H))
+    got, ref = [], []
+    for b in range(B):
+        for h in range(H):
+            u = b * H + h
+            s1 = np.nonzero(active[:T1, b])[0]
+            s2 = np.arange(T1, T)
+            S_start = S0[b, h].double().numpy()[None]
+            if len(s1):
+                r1 = oracle.run(p, S_start, q[u:u + 1, s1], k[u:u + 1, s1], v[u:u + 1, s1], g[u:u + 1, s1],
+                                beta[u:u + 1, s1], snapshots=False)
+                ref.append(r1.o[0])
+                got.append(o_gpu[s1, b, h])
+                S_start = r1.S_final          # the pending flush encodes the window where it stands
+            r2 = oracle.run(p, S_start, q[u:u + 1, s2], k[u:u + 1, s2], v[u:u + 1, s2], g[u:u + 1, s2],
+                            beta[u:u + 1, s2], snapshots=False)
+            ref.append(r2.o[0])
+            got.append(o_gpu[s2, b, h])
+    err = rel_l2(np.concatenate(got), np.concatenate(ref))
+    assert err <= 1e-3, err
