@@ -732,6 +732,66 @@ def ragged_phases(dev, wl, L: int = 4, reps: int = 20) -> list[dict]:
     return rows
 
 
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12     # FP32 FMA lanes x 2 FLOP x max SM clock
+
+
+def prefill_timing(dev, wl, T: int | None = None, reps: int = 5) -> list[dict]:
+    """A prompt of T tokens for every sequence (default: the workload's prefill
+    length) from a zero state to the encoded window-start state, with every
+    prompt token's output: lq_prefill_tokens (register-resident FP32
+    recurrence plus codec, one launch) against the route through the decode
+    kernels (T FP32-state decode launches, then lq_prefill_state)."""
+    from recurrent_state_quantization_lq_b200 import lq
+    T = T or wl.prefill_tokens
+    B, H, d = wl.batch, wl.heads, wl.d_k
+    gate = "channel" if wl.per_channel_gate else "scalar"
+    tb = inputs.tokens_on_device(wl.seed * 100 + 77, T, B, H, d, d, wl.per_channel_gate, wl.dtype, dev)
+    out = torch.empty(T, B, H, d, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    win = lq.DecodeState(B, H, d, window=wl.window, n_comp_rows=wl.n_comp_rows, n_comp_cols=wl.n_comp_cols,
+                         gate=gate, in_dtype=wl.dtype, device=dev)
+    f32 = lq.DecodeState(B, H, d, gate=gate, mode="fp32", in_dtype=wl.dtype, device=dev)
+
+    def fused():
+        win.prefill_tokens(tb.q, tb.k, tb.v, tb.g, tb.beta, out=out)
+
+    def token_loop():
+        f32.prefill(None)
+        for t in range(T):
+            f32.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=out[t])
+        win.prefill(f32.view("state_f32"))
+
+    rows = []
+    flop = (6 + (1 if wl.per_channel_gate else 0)) * d * d          # per token and head
+    for name, fn in (("prefill_tokens", fused), ("decode_loop", token_loop)):
+        with torch.cuda.stream(stream):
+            fn()                                                    # warm (kernel attributes)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        assert win.device_status(stream) == lq.LQ_OK, lq.last_error()
+        ms = e0.elapsed_time(e1) / reps
+        tflops = B * H * T * flop / (ms * 1e-3) / 1e12
+        rows.append({"path": name, "workload": wl.name, "batch": B, "heads": H, "d": d, "prompt_tokens": T,
+                     "ms": ms, "prompt_tokens_per_s_per_layer": B * T / (ms * 1e-3),
+                     "recurrence_tflops": tflops, "frac_of_fp32_simt_peak": tflops / FP32_SIMT_TFLOPS,
+                     "launches": 1 if name == "prefill_tokens" else T + 1})
+        del g
+    rows.append({"path": "speedup", "value": rows[1]["ms"] / rows[0]["ms"]})
+    return rows
+
+
 def quality_study(dev, tokens: int = 1024) -> list[dict]:
     """Output error against the FP32 state over window sizes and compensator
     counts (16 sequences x 32 heads, 128 x 128), on the planted-outlier start
@@ -802,6 +862,9 @@ def main():
                     help="print one JSON line per (start state, W, n_c) point of the output-error study")
     ap.add_argument("--ragged", nargs="?", const="gdn_b64_h32_d128_w64", default=None, metavar="WORKLOAD",
                     help="print one JSON line per variant of the staggered-phase (continuous batching) timing")
+    ap.add_argument("--prefill", nargs="?", const="gdn_b64_h32_d128_w64", default=None, metavar="WORKLOAD",
+                    help="time the prompt prefill (lq_prefill_tokens against per-token decode launches)")
+    ap.add_argument("--prefill-tokens", type=int, default=None)
     ap.add_argument("--sweep", action="store_true",
                     help="print one JSON line per point of the batch x window throughput sweep instead of timing")
     args = ap.parse_args()
@@ -820,6 +883,12 @@ def main():
         torch.cuda.set_device(0)
         for row in quality_study(torch.device("cuda", 0)):
             print(json.dumps({"mode": "quality_study", **row}), flush=True)
+        return
+
+    if args.prefill is not None:
+        torch.cuda.set_device(0)
+        for row in prefill_timing(torch.device("cuda", 0), inputs.WORKLOADS[args.prefill], args.prefill_tokens):
+            print(json.dumps({"mode": "prefill", **row}), flush=True)
         return
 
     if args.ragged is not None:

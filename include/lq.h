@@ -220,6 +220,30 @@ LQ_API lq_status lq_window_flush_pending(lq_handle h, void *stream);
  */
 LQ_API lq_status lq_prefill_sequences(lq_handle h, const float *d_S0, const uint8_t *d_mask, void *stream);
 
+/*
+ * Prefill from prompt tokens: run the FP32 recurrence of the gated delta rule
+ * over n_tokens prompt tokens of every sequence, starting from d_S0 (device
+ * FP32 [batch][heads][d_v][d_k]; NULL = all-zero state), and make the state
+ * after the last token the window-start state, exactly as lq_prefill_state()
+ * would from that FP32 state: encoded (windowed and naive modes) or stored
+ * (FP32 mode).  The prompt runs at full precision; the codec of LeapQuant
+ * ("LeapQuant: Efficient Linear Attention with Accurate Recurrent State
+ * Quantization", section "Abstract (arXiv)") applies once, at its end.
+ * Inputs are token-major, each token laid out as for lq_decode_step():
+ *   d_q, d_k, d_v: in_dtype [n_tokens][batch][heads][d]  (16-byte aligned);
+ *   d_g: f32 [n_tokens][batch][heads] (GDN) or [..][d_k] (KDA, 16-byte aligned);
+ *   d_beta: f32 [n_tokens][batch][heads].
+ * d_o: f32 [n_tokens][batch][heads][d_v], o_t = S_t q_t for every prompt
+ * token, or NULL to skip the outputs.  n_tokens = 0 is lq_prefill_state().
+ * Afterwards every window is empty (ragged handles: every count is 0 and the
+ * phases are aligned).  The caller keeps ownership of every buffer; nothing is
+ * retained after the call.  Errors: LQ_ERR_INVALID_ARG for a NULL input with
+ * n_tokens > 0, a negative n_tokens or a misaligned pointer.
+ */
+LQ_API lq_status lq_prefill_tokens(lq_handle h, const float *d_S0, const void *d_q, const void *d_k,
+                                   const void *d_v, const float *d_g, const float *d_beta, int32_t n_tokens,
+                                   float *d_o, void *stream);
+
 /* Tokens buffered in the current window (0..W); -1 for a bad or ragged handle
  * (a ragged handle's counts are on the device, at lq_layout.fill). */
 LQ_API int32_t lq_window_fill(lq_handle h);

@@ -249,6 +249,45 @@ lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream) {
     return LQ_OK;
 }
 
+lq_status lq_prefill_tokens(lq_handle h, const float *d_S0, const void *d_q, const void *d_k, const void *d_v,
+                            const float *d_g, const float *d_beta, int32_t n_tokens, float *d_o, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    if (n_tokens < 0) return fail(LQ_ERR_INVALID_ARG, "negative n_tokens");
+    if (n_tokens == 0) return lq_prefill_state(h, d_S0, stream);
+    const lq_config &c = h->cfg;
+    if (!d_q || !d_k || !d_v || !d_g || !d_beta) return fail(LQ_ERR_INVALID_ARG, "NULL prompt input");
+    if (!aligned(d_q, 16) || !aligned(d_k, 16) || !aligned(d_v, 16))
+        return fail(LQ_ERR_INVALID_ARG, "q, k, v must be 16-byte aligned");
+    if (!aligned(d_g, c.gate == LQ_GATE_CHANNEL ? 16 : 4) || !aligned(d_beta, 4) || (d_o && !aligned(d_o, 4)))
+        return fail(LQ_ERR_INVALID_ARG, "g, beta, o misaligned (g per-channel: 16 bytes; others: 4)");
+    if (d_S0 != nullptr && !aligned(d_S0, 16)) return fail(LQ_ERR_INVALID_ARG, "S0 must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    lq::Views v = views(h);
+    cudaError_t e = cudaMemsetAsync(v.err, 0, 256, s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+    lq::TokenPrefillArgs a;
+    a.w = v;
+    a.S0 = d_S0;
+    a.q = d_q; a.k = d_k; a.v = d_v; a.g = d_g; a.beta = d_beta; a.o = d_o;
+    a.n_tokens = n_tokens;
+    const bool win = (c.mode == LQ_MODE_WINDOW);
+    a.n_rows = win ? c.n_comp_rows : 0;
+    a.n_cols = win ? c.n_comp_cols : 0;
+    a.smooth = win ? c.smooth : 0;
+    a.select = win ? c.select : LQ_SELECT_L2;
+    a.fp32_state = (c.mode == LQ_MODE_FP32);
+    e = lq::launch_prefill_tokens(a, c.d_k, c.gate, c.in_dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "launching the token prefill kernel");
+    if (c.ragged) {
+        e = cudaMemsetAsync(h->ws + h->lay.fill, 0, (size_t)c.batch * c.heads * 4, s);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the window counts");
+    }
+    h->n_buf = 0;
+    h->prefilled = 1;
+    h->aligned = 1;
+    return LQ_OK;
+}
+
 namespace {
 
 lq_status decode_impl(lq_handle h, const void *d_q, const void *d_k, const void *d_v, const float *d_g,

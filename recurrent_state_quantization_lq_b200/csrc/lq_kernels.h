@@ -41,6 +41,23 @@ struct DecodeArgs {
     int heads;         // units per sequence
 };
 
+struct TokenPrefillArgs {
+    Views w;
+    const float *S0;   // starting state [N][d][d], or nullptr for zeros
+    const void *q;     // prompt inputs [T][N][d] (in_dtype)
+    const void *k;
+    const void *v;
+    const float *g;    // log alpha [T][N] (GDN) or [T][N][d] (KDA)
+    const float *beta; // [T][N]
+    float *o;          // outputs [T][N][d], or nullptr
+    int n_tokens;      // T
+    int n_rows;        // compensator rows to extract
+    int n_cols;        // compensator columns to extract
+    int smooth;        // column smoothing on/off
+    int select;        // LQ_SELECT_*
+    int fp32_state;    // 1: store the FP32 state (FP32 mode) instead of encoding it
+};
+
 // Encode the tensor map the windowed decode uses to load one unit's INT8 tile
 // (d x d, 128- or 64-byte swizzle) from `codes` ([units][d][d]).  Host only.
 cudaError_t make_codes_map(void *map_out, const int8_t *codes, int d, int units);
@@ -48,6 +65,7 @@ cudaError_t make_codes_map(void *map_out, const int8_t *codes, int d, int units)
 // d = d_k = d_v in {64, 128}; gate: LQ_GATE_*; in_dtype: LQ_DTYPE_*.
 cudaError_t launch_encode(const EncodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
 cudaError_t launch_flush_split(const EncodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
+cudaError_t launch_prefill_tokens(const TokenPrefillArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
 cudaError_t launch_decode_window(const DecodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
 cudaError_t launch_decode_fp32(const DecodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);
 cudaError_t launch_decode_naive(const DecodeArgs &a, int d, int gate, int in_dtype, cudaStream_t s);

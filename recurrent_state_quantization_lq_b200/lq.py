@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.lq_window_flush_pending.restype = i32
         L.lq_prefill_sequences.argtypes = [vp, vp, vp, vp]
         L.lq_prefill_sequences.restype = i32
+        L.lq_prefill_tokens.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
+        L.lq_prefill_tokens.restype = i32
         L.lq_window_fill.argtypes = [vp]
         L.lq_window_fill.restype = i32
         L.lq_device_status.argtypes = [vp, vp]
@@ -213,6 +215,26 @@ class DecodeState:
         assert mask.dtype == torch.uint8 and mask.numel() == self.batch and mask.device == self.device
         self._check(lib().lq_prefill_sequences(self._h, _ptr(S0), _ptr(mask), _stream_ptr(stream, self.device)),
                     "lq_prefill_sequences")
+
+    def prefill_tokens(self, q, k, v, g, beta, S0: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor | None:
+        """Run the FP32 recurrence over a prompt (inputs [T, batch, heads, ...]
+        as for decode_step, stacked over tokens) from S0 (None = zero state) and
+        encode its final state as the window-start state.  Writes the prompt's
+        outputs into `out` ([T, batch, heads, d] FP32) when given."""
+        T = q.shape[0]
+        for t, dt in ((q, self.in_dtype), (k, self.in_dtype), (v, self.in_dtype), (g, torch.float32),
+                      (beta, torch.float32)):
+            assert t.dtype == dt and t.is_contiguous() and t.device == self.device and t.shape[0] == T, t.dtype
+        if out is not None:
+            assert out.dtype == torch.float32 and out.is_contiguous() and out.device == self.device
+            assert out.numel() == T * self.batch * self.heads * self.d
+        if S0 is not None:
+            assert S0.dtype == torch.float32 and S0.is_contiguous() and S0.device == self.device
+            assert S0.numel() == self.batch * self.heads * self.d * self.d
+        self._check(lib().lq_prefill_tokens(self._h, _ptr(S0), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), T,
+                                            _ptr(out), _stream_ptr(stream, self.device)), "lq_prefill_tokens")
+        return out
 
     @property
     def fill(self) -> int:

@@ -1,12 +1,15 @@
 """Run a short, fixed sequence of liblq launches for a profiler to capture.
 
     python -m recurrent_state_quantization_lq_b200.profile_case [--workload NAME]
-        [--mode window|fp32|naive] [--tokens T] [--flush]
+        [--mode window|fp32|naive] [--tokens T] [--flush] [--prompt P] [--batch B]
 
 Sets up one layer-state of the workload (prefill from a seeded FP32 state),
 then runs T decode launches (the windowed kernel sees 0..T-1 buffered tokens)
 and, with --flush, one window flush.  Launch order: the prefill's encode
 launch (windowed/naive modes), then the T decode launches, then the flush.
+With --prompt P the state is instead prefilled from a P-token prompt by one
+token-prefill launch (lq_prefill_tokens).  --batch overrides the workload's
+batch (smaller captures).
 """
 from __future__ import annotations
 
@@ -23,8 +26,14 @@ def main() -> None:
     ap.add_argument("--mode", default="window", choices=["window", "fp32", "naive"])
     ap.add_argument("--tokens", type=int, default=34)
     ap.add_argument("--flush", action="store_true")
+    ap.add_argument("--prompt", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=0)
     args = ap.parse_args()
     wl = inputs.WORKLOADS[args.workload]
+    if args.batch:
+        wl = inputs.Workload(wl.name, args.batch, wl.heads, wl.d_k, wl.d_v, wl.window, wl.n_comp_rows,
+                             wl.n_comp_cols, wl.per_channel_gate, wl.prefill_tokens, wl.decode_tokens, wl.dtype,
+                             wl.seed, planted=wl.planted)
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     T = min(args.tokens, wl.window) if args.mode == "window" else args.tokens
@@ -34,7 +43,13 @@ def main() -> None:
     st = lq.DecodeState(wl.batch, wl.heads, wl.d_k, window=wl.window, n_comp_rows=wl.n_comp_rows,
                         n_comp_cols=wl.n_comp_cols, gate="channel" if wl.per_channel_gate else "scalar",
                         mode=args.mode, in_dtype=wl.dtype, device=dev)
-    st.prefill(S0)
+    if args.prompt:
+        pb = inputs.tokens_on_device(wl.seed + 1, args.prompt, wl.batch, wl.heads, wl.d_k, wl.d_v,
+                                     wl.per_channel_gate, wl.dtype, dev)
+        po = torch.empty(args.prompt, wl.batch, wl.heads, wl.d_v, dtype=torch.float32, device=dev)
+        st.prefill_tokens(pb.q, pb.k, pb.v, pb.g, pb.beta, S0=S0, out=po)
+    else:
+        st.prefill(S0)
     out = torch.empty(wl.batch, wl.heads, wl.d_v, dtype=torch.float32, device=dev)
     for t in range(T):
         st.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=out)
@@ -43,7 +58,8 @@ def main() -> None:
     status = st.device_status()
     if status != lq.LQ_OK:
         raise lq.LQError(status, "profile_case")
-    print(f"profile_case: {wl.name} mode={args.mode} tokens={T} flush={args.flush} ok")
+    print(f"profile_case: {wl.name} batch={wl.batch} mode={args.mode} prompt={args.prompt} tokens={T} "
+          f"flush={args.flush} ok")
 
 
 if __name__ == "__main__":

@@ -13,7 +13,8 @@ def test_exports_every_declared_symbol():
     assert set(names) >= {"lq_workspace_bytes", "lq_workspace_layout", "lq_state_create",
                           "lq_prefill_state", "lq_decode_step", "lq_window_flush", "lq_window_fill",
                           "lq_device_status", "lq_state_destroy", "lq_last_error_string",
-                          "lq_decode_step_active", "lq_window_flush_pending", "lq_prefill_sequences"}
+                          "lq_decode_step_active", "lq_window_flush_pending", "lq_prefill_sequences",
+                          "lq_prefill_tokens"}
     L = lq.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -138,3 +139,21 @@ def test_ragged_entry_points_check_the_handle_kind():
     assert L.lq_decode_step_active(ragged, p, p, p, p, p, None, p, None) == lq.LQ_ERR_STATE
     assert L.lq_state_destroy(shared) == lq.LQ_OK
     assert L.lq_state_destroy(ragged) == lq.LQ_OK
+
+
+def test_prefill_tokens_validates_on_the_host():
+    L = lq.lib()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: every call below returns before any launch
+    h = ctypes.c_void_p()
+    cfg = lq.make_config(2, 3, 64, window=8, gate="channel")
+    assert L.lq_state_create(ctypes.byref(cfg), fake, lq.workspace_bytes(cfg), ctypes.byref(h)) == lq.LQ_OK
+    p = ctypes.c_void_p(1 << 21)
+    assert L.lq_prefill_tokens(h, None, p, p, p, p, p, -1, None, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_prefill_tokens(h, None, None, p, p, p, p, 4, None, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_prefill_tokens(h, None, p, p, p, None, p, 4, None, None) == lq.LQ_ERR_INVALID_ARG
+    odd = ctypes.c_void_p((1 << 21) + 8)
+    assert L.lq_prefill_tokens(h, None, odd, p, p, p, p, 4, None, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_prefill_tokens(h, None, p, p, p, odd, p, 4, None, None) == lq.LQ_ERR_INVALID_ARG   # KDA gate: 16 B
+    assert L.lq_prefill_tokens(h, odd, p, p, p, p, p, 4, None, None) == lq.LQ_ERR_INVALID_ARG     # S0: 16 B
+    assert L.lq_prefill_tokens(None, None, p, p, p, p, p, 4, None, None) == lq.LQ_ERR_INVALID_ARG
+    assert L.lq_state_destroy(h) == lq.LQ_OK
