@@ -244,6 +244,26 @@ LQ_API lq_status lq_prefill_tokens(lq_handle h, const float *d_S0, const void *d
                                    const void *d_v, const float *d_g, const float *d_beta, int32_t n_tokens,
                                    float *d_o, void *stream);
 
+/*
+ * Ragged handles: start new sequences in some batch slots from their prompts,
+ * as lq_prefill_sequences() does from a state.  The sequences with
+ * d_mask[b] != 0 (device uint8 [batch]) run the FP32 recurrence from d_S0
+ * (their rows; NULL = zero state) over their first d_lengths[b] prompt tokens
+ * (device int32 [batch], clamped to 0..max_tokens; NULL = max_tokens for
+ * all), and the state after them is encoded as their window-start state, with
+ * their windows emptied.  Prompt inputs are laid out as for
+ * lq_prefill_tokens() over max_tokens tokens; only the rows of masked
+ * sequences and of their own tokens are read, and only those outputs are
+ * written (d_o may be NULL).  Other sequences are untouched.  Requires a prior
+ * lq_prefill_state(); LQ_ERR_STATE on a shared-phase handle; LQ_ERR_INVALID_ARG
+ * for a NULL mask, a negative max_tokens, a NULL input with max_tokens > 0 or a
+ * misaligned pointer.
+ */
+LQ_API lq_status lq_prefill_sequences_tokens(lq_handle h, const float *d_S0, const void *d_q, const void *d_k,
+                                             const void *d_v, const float *d_g, const float *d_beta,
+                                             int32_t max_tokens, const int32_t *d_lengths, const uint8_t *d_mask,
+                                             float *d_o, void *stream);
+
 /* Tokens buffered in the current window (0..W); -1 for a bad or ragged handle
  * (a ragged handle's counts are on the device, at lq_layout.fill). */
 LQ_API int32_t lq_window_fill(lq_handle h);

@@ -276,6 +276,10 @@ lq_status lq_prefill_tokens(lq_handle h, const float *d_S0, const void *d_q, con
     a.smooth = win ? c.smooth : 0;
     a.select = win ? c.select : LQ_SELECT_L2;
     a.fp32_state = (c.mode == LQ_MODE_FP32);
+    a.seq_mask = nullptr;
+    a.lengths = nullptr;
+    a.heads = c.heads;
+    a.fill = nullptr;                     // every count is cleared below
     e = lq::launch_prefill_tokens(a, c.d_k, c.gate, c.in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "launching the token prefill kernel");
     if (c.ragged) {
@@ -285,6 +289,44 @@ lq_status lq_prefill_tokens(lq_handle h, const float *d_S0, const void *d_q, con
     h->n_buf = 0;
     h->prefilled = 1;
     h->aligned = 1;
+    return LQ_OK;
+}
+
+lq_status lq_prefill_sequences_tokens(lq_handle h, const float *d_S0, const void *d_q, const void *d_k,
+                                      const void *d_v, const float *d_g, const float *d_beta, int32_t max_tokens,
+                                      const int32_t *d_lengths, const uint8_t *d_mask, float *d_o, void *stream) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    const lq_config &c = h->cfg;
+    if (!c.ragged) return fail(LQ_ERR_STATE, "lq_prefill_sequences_tokens needs a ragged handle");
+    if (!h->prefilled) return fail(LQ_ERR_STATE, "lq_prefill_sequences_tokens before lq_prefill_state");
+    if (d_mask == nullptr) return fail(LQ_ERR_INVALID_ARG, "NULL sequence mask");
+    if (max_tokens < 0) return fail(LQ_ERR_INVALID_ARG, "negative max_tokens");
+    if (max_tokens > 0) {
+        if (!d_q || !d_k || !d_v || !d_g || !d_beta) return fail(LQ_ERR_INVALID_ARG, "NULL prompt input");
+        if (!aligned(d_q, 16) || !aligned(d_k, 16) || !aligned(d_v, 16))
+            return fail(LQ_ERR_INVALID_ARG, "q, k, v must be 16-byte aligned");
+        if (!aligned(d_g, c.gate == LQ_GATE_CHANNEL ? 16 : 4) || !aligned(d_beta, 4) || (d_o && !aligned(d_o, 4)))
+            return fail(LQ_ERR_INVALID_ARG, "g, beta, o misaligned (g per-channel: 16 bytes; others: 4)");
+    }
+    if (d_lengths != nullptr && !aligned(d_lengths, 4)) return fail(LQ_ERR_INVALID_ARG, "lengths misaligned");
+    if (d_S0 != nullptr && !aligned(d_S0, 16)) return fail(LQ_ERR_INVALID_ARG, "S0 must be 16-byte aligned");
+    lq::TokenPrefillArgs a;
+    a.w = views(h);
+    a.S0 = d_S0;
+    a.q = d_q; a.k = d_k; a.v = d_v; a.g = d_g; a.beta = d_beta; a.o = d_o;
+    a.n_tokens = max_tokens;
+    a.n_rows = c.n_comp_rows;
+    a.n_cols = c.n_comp_cols;
+    a.smooth = c.smooth;
+    a.select = c.select;
+    a.fp32_state = 0;
+    a.seq_mask = d_mask;
+    a.lengths = d_lengths;
+    a.heads = c.heads;
+    a.fill = reinterpret_cast<int32_t *>(h->ws + h->lay.fill);
+    cudaError_t e = lq::launch_prefill_tokens(a, c.d_k, c.gate, c.in_dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launching the token prefill kernel");
+    h->aligned = 0;                       // the restarted sequences start a new phase
     return LQ_OK;
 }
 

@@ -56,6 +56,12 @@ struct TokenPrefillArgs {
     int smooth;        // column smoothing on/off
     int select;        // LQ_SELECT_*
     int fp32_state;    // 1: store the FP32 state (FP32 mode) instead of encoding it
+    // ragged restarts: sequences to prefill (null: all), per-sequence prompt
+    // lengths <= n_tokens (null: n_tokens), units per sequence, counts to clear
+    const uint8_t *seq_mask;
+    const int32_t *lengths;
+    int heads;
+    int32_t *fill;
 };
 
 // Encode the tensor map the windowed decode uses to load one unit's INT8 tile

@@ -114,7 +114,9 @@ __global__ void __launch_bounds__(kTile, 2) prefill_tokens_kernel(TokenPrefillAr
     const int cg = lane % LPR;                                       // column piece index in the row block
     const int r0 = (tid / LPR) * 4;                                  // the block's first row
     const int lane0 = lane - cg;                                     // the row block's first lane
-    const int units = a.w.units, T = a.n_tokens;
+    const int units = a.w.units, b = u / a.heads;
+    if (a.seq_mask != nullptr && a.seq_mask[b] == 0) return;       // sequence not restarted
+    const int T = a.lengths != nullptr ? min(max(a.lengths[b], 0), a.n_tokens) : a.n_tokens;
     auto col = [&](int m) { return m * 4 * LPR + cg * 4; };          // first of 4 owned columns in piece m
     // after the butterfly this lane holds the sum of row r0 + mine
     const bool hb = (cg & (LPR / 2)) != 0, lb = (cg & (LPR / 4)) != 0;
@@ -324,6 +326,7 @@ __global__ void __launch_bounds__(kTile, 2) prefill_tokens_kernel(TokenPrefillAr
             *reinterpret_cast<float4 *>(ps + (r0 + i) * D + col(m)) =
                 make_float4(S[i][m][0].x, S[i][m][0].y, S[i][m][1].x, S[i][m][1].y);
     __syncthreads();
+    if (a.fill != nullptr && tid == 0) a.fill[u] = 0;                // the unit's window starts empty
     constexpr int G = Tile<D>::G, NR = Tile<D>::NR;
     Tile<D> Tl;
     Tl.tid = tid;

@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.lq_prefill_sequences.restype = i32
         L.lq_prefill_tokens.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
         L.lq_prefill_tokens.restype = i32
+        L.lq_prefill_sequences_tokens.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
+        L.lq_prefill_sequences_tokens.restype = i32
         L.lq_window_fill.argtypes = [vp]
         L.lq_window_fill.restype = i32
         L.lq_device_status.argtypes = [vp, vp]
@@ -234,6 +236,31 @@ class DecodeState:
             assert S0.numel() == self.batch * self.heads * self.d * self.d
         self._check(lib().lq_prefill_tokens(self._h, _ptr(S0), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), T,
                                             _ptr(out), _stream_ptr(stream, self.device)), "lq_prefill_tokens")
+        return out
+
+    def prefill_sequences_tokens(self, q, k, v, g, beta, mask: torch.Tensor, lengths: torch.Tensor | None = None,
+                                 S0: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                                 stream=None) -> torch.Tensor | None:
+        """Ragged: restart the sequences with mask[b] != 0 from S0 (None = zero)
+        through their prompts: inputs [T, batch, heads, ...] padded to T tokens,
+        lengths int32 [batch] on the device (None = T for every sequence)."""
+        T = q.shape[0]
+        for t, dt in ((q, self.in_dtype), (k, self.in_dtype), (v, self.in_dtype), (g, torch.float32),
+                      (beta, torch.float32)):
+            assert t.dtype == dt and t.is_contiguous() and t.device == self.device and t.shape[0] == T, t.dtype
+        assert mask.dtype == torch.uint8 and mask.numel() == self.batch and mask.device == self.device
+        if lengths is not None:
+            assert lengths.dtype == torch.int32 and lengths.numel() == self.batch and lengths.device == self.device
+        if out is not None:
+            assert out.dtype == torch.float32 and out.is_contiguous() and out.device == self.device
+            assert out.numel() == T * self.batch * self.heads * self.d
+        if S0 is not None:
+            assert S0.dtype == torch.float32 and S0.is_contiguous() and S0.device == self.device
+            assert S0.numel() == self.batch * self.heads * self.d * self.d
+        self._check(lib().lq_prefill_sequences_tokens(self._h, _ptr(S0), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                                      _ptr(beta), T, _ptr(lengths), _ptr(mask), _ptr(out),
+                                                      _stream_ptr(stream, self.device)),
+                    "lq_prefill_sequences_tokens")
         return out
 
     @property

@@ -14,7 +14,7 @@ def test_exports_every_declared_symbol():
                           "lq_prefill_state", "lq_decode_step", "lq_window_flush", "lq_window_fill",
                           "lq_device_status", "lq_state_destroy", "lq_last_error_string",
                           "lq_decode_step_active", "lq_window_flush_pending", "lq_prefill_sequences",
-                          "lq_prefill_tokens"}
+                          "lq_prefill_tokens", "lq_prefill_sequences_tokens"}
     L = lq.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -131,11 +131,13 @@ def test_ragged_entry_points_check_the_handle_kind():
     # shared-phase handles refuse the ragged calls
     assert L.lq_decode_step_active(shared, p, p, p, p, p, None, p, None) == lq.LQ_ERR_STATE
     assert L.lq_prefill_sequences(shared, None, p, None) == lq.LQ_ERR_STATE
+    assert L.lq_prefill_sequences_tokens(shared, None, p, p, p, p, p, 4, None, p, None, None) == lq.LQ_ERR_STATE
     # ragged handles: counts live on the device; order of calls is checked on the host
     assert L.lq_window_fill(ragged) == -1
     assert L.lq_window_fill(shared) == 0
     assert L.lq_prefill_sequences(ragged, None, p, None) == lq.LQ_ERR_STATE      # before lq_prefill_state
     assert L.lq_window_flush_pending(ragged, None) == lq.LQ_ERR_STATE            # before lq_prefill_state
+    assert L.lq_prefill_sequences_tokens(ragged, None, p, p, p, p, p, 4, None, p, None, None) == lq.LQ_ERR_STATE
     assert L.lq_decode_step_active(ragged, p, p, p, p, p, None, p, None) == lq.LQ_ERR_STATE
     assert L.lq_state_destroy(shared) == lq.LQ_OK
     assert L.lq_state_destroy(ragged) == lq.LQ_OK

@@ -203,3 +203,70 @@ def test_ragged_phases_realign_after_flush_pending():
             got.append(o_gpu[s2, b, h])
     err = rel_l2(np.concatenate(got), np.concatenate(ref))
     assert err <= 1e-3, err
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_ragged_restart_from_prompts_of_different_lengths(gate):
+    """Sequences 1 and 3 restart mid-stream from their own prompts (lengths 5
+    and 0 of a 7-token padded batch); each restarted unit follows the oracle's
+    FP32 recurrence over its prompt, the encoded result, then the windowed run
+    over its later tokens.  The other sequences are untouched."""
+    d, B, H, W, T, J, P = 64, 4, 2, 5, 18, 9, 7
+    lengths = np.array([7, 5, 3, 0], dtype=np.int32)
+    mask = np.array([0, 1, 0, 1], dtype=np.uint8)
+    per_channel = gate == "channel"
+    tb = inputs.tokens(71, 0, T, B, H, d, d, per_channel)
+    pb = inputs.tokens(72, 0, P, B, H, d, d, per_channel)
+    rng = np.random.default_rng(71)
+    active = rng.random((T, B)) < 0.75
+    gen = torch.Generator().manual_seed(71)
+    S0 = 0.5 * torch.randn(B, H, d, d, generator=gen)
+    S1 = 0.5 * torch.randn(B, H, d, d, generator=gen)
+    st = lq.DecodeState(B, H, d, window=W, n_comp_rows=1, n_comp_cols=1, gate=gate, ragged=True, device=DEV)
+    st.prefill(S0.to(DEV).contiguous())
+    tbd, pbd = to_device(tb, DEV), to_device(pb, DEV)
+    out = torch.full((T, B, H, d), float("nan"), device=DEV)
+    pout = torch.full((P, B, H, d), float("nan"), device=DEV)
+    for t in range(T):
+        if t == J:
+            st.prefill_sequences_tokens(pbd.q, pbd.k, pbd.v, pbd.g, pbd.beta,
+                                        torch.tensor(mask, device=DEV), torch.tensor(lengths, device=DEV),
+                                        S0=S1.to(DEV).contiguous(), out=pout)
+        act = torch.tensor(active[t].astype(np.uint8), device=DEV)
+        st.decode_step(tbd.q[t], tbd.k[t], tbd.v[t], tbd.g[t], tbd.beta[t], out=out[t], active=act)
+        st.flush()
+    assert st.device_status() == lq.LQ_OK, lq.last_error()
+    o_gpu, p_gpu = out.cpu().numpy(), pout.cpu().numpy()
+    pw = oracle_params(d, W, 1, 1, gate, "window")
+    pf = oracle_params(d, W, 1, 1, gate, "fp32")
+    q, k, v, g, beta = unit_inputs(tb, range(B * H))
+    pq, pk, pv, pg, pbeta = unit_inputs(pb, range(B * H))
+    got, ref, pgot, pref = [], [], [], []
+    for b in range(B):
+        for h in range(H):
+            u = b * H + h
+            steps = np.nonzero(active[:, b])[0]
+            segs = [(S0[b, h].double().numpy()[None], steps)]
+            if mask[b]:
+                L = int(lengths[b])
+                S_start = S1[b, h].double().numpy()[None]
+                if L:
+                    rp = oracle.run(pf, S_start, pq[u:u + 1, :L], pk[u:u + 1, :L], pv[u:u + 1, :L],
+                                    pg[u:u + 1, :L], pbeta[u:u + 1, :L], snapshots=False)
+                    pref.append(rp.o[0])
+                    pgot.append(p_gpu[:L, b, h])
+                    S_start = rp.S_final
+                assert np.isnan(p_gpu[L:, b, h]).all()
+                segs = [(segs[0][0], steps[steps < J]), (S_start, steps[steps >= J])]
+            else:
+                assert np.isnan(p_gpu[:, b, h]).all()
+            for S_s, seg in segs:
+                if len(seg) == 0:
+                    continue
+                r = oracle.run(pw, S_s, q[u:u + 1, seg], k[u:u + 1, seg], v[u:u + 1, seg], g[u:u + 1, seg],
+                               beta[u:u + 1, seg], snapshots=False)
+                ref.append(r.o[0])
+                got.append(o_gpu[seg, b, h])
+    assert rel_l2(np.concatenate(pgot), np.concatenate(pref)) <= 1e-5
+    err = rel_l2(np.concatenate(got), np.concatenate(ref))
+    assert err <= 1e-3, err
