@@ -69,6 +69,7 @@ struct TokShape {
     static constexpr int WORDS_CODEC = D * D;      // the final state, row-major (the codec scratch reuses it)
     static constexpr int WORDS = WORDS_STAGES > WORDS_CODEC ? WORDS_STAGES : WORDS_CODEC;
     static_assert(CodecScratch<D>::FLOATS <= WORDS_CODEC, "codec scratch fits");
+    static_assert(2 * kTokChunk <= NT && kTokChunk <= NT, "gate and beta copies");
     static_assert(RQ % 4 == 0 && RV % 4 == 0 && RG % 4 == 0 && RB % 4 == 0, "16-byte aligned");
 };
 
@@ -169,10 +170,10 @@ __global__ void __launch_bounds__(kTile, 2) prefill_tokens_kernel(TokenPrefillAr
             }
             if (tid < ne) cp_async4(ps + Sh::RB + tid, a.beta + (size_t)(t0 + tid) * units + u);
         } else {
-            const int e = tid & 15;
-            if (tid < 32 && e < ne)
-                cp_async4(ps + (tid < 16 ? Sh::RG : Sh::RB) + e,
-                          (tid < 16 ? a.g : a.beta) + (size_t)(t0 + e) * units + u);
+            const int e = tid % kTokChunk;
+            if (tid < 2 * kTokChunk && e < ne)
+                cp_async4(ps + (tid < kTokChunk ? Sh::RG : Sh::RB) + e,
+                          (tid < kTokChunk ? a.g : a.beta) + (size_t)(t0 + e) * units + u);
         }
     };
     // pass 1: the gate products c_t and 1/c_t of every channel (serial over the chunk)
