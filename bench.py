@@ -272,17 +272,16 @@ class LayerStack:
 
 
 def fp32_prefill(wl, n_layers, device, seed):
-    """Per layer: the FP32 recurrence over the workload's prefill tokens from zero."""
+    """Per layer: the FP32 recurrence over the workload's prefill tokens from
+    zero (one lq_prefill_tokens launch on an FP32-state handle)."""
     from recurrent_state_quantization_lq_b200 import lq
     gate = "channel" if wl.per_channel_gate else "scalar"
     S = []
     for l in range(n_layers):
         st = lq.DecodeState(wl.batch, wl.heads, wl.d_k, gate=gate, mode="fp32", in_dtype=wl.dtype, device=device)
-        st.prefill(None)
         tb = inputs.tokens_on_device(seed * 100 + 50 + l, wl.prefill_tokens, wl.batch, wl.heads, wl.d_k, wl.d_v,
                                      wl.per_channel_gate, wl.dtype, device)
-        for t in range(wl.prefill_tokens):
-            st.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t])
+        st.prefill_tokens(tb.q, tb.k, tb.v, tb.g, tb.beta)
         S.append(st.view("state_f32").clone())
         del st, tb
     torch.cuda.synchronize()
