@@ -306,7 +306,11 @@ __global__ void __launch_bounds__(kThreads) flush_split_kernel(EncodeArgs a) {
                 float *csq = fs + Sh::CSQ + parity * C * D, *cmx = fs + Sh::CMX + parity * C * D;
                 int32_t *cidx = w.comp_index + (size_t)u * cis;
 
+                // Every global store of the unit waits until after the last cluster
+                // barrier: a barrier's release would otherwise wait for them to drain.
                 // 2a. compensator rows: every CTA sends its 16 row scores to every CTA
+                uint2 sel = make_uint2(0xffffffffu, 0xffffffffu);
+                int rslot[4] = {-1, -1, -1, -1};          // compensator slot of each of this thread's rows
                 if (ncr > 0) {
                     float pr[4];
 #pragma unroll
@@ -325,39 +329,23 @@ __global__ void __launch_bounds__(kThreads) flush_split_kernel(EncodeArgs a) {
                         cluster.map_shared_rank(rsc, (unsigned)(lane >> 2))[row0 + i] = v;
                     }
                     cluster.sync();
-                    const uint2 sel = select_top<D>(rsc, ncr);
-                    if (rank == 0 && tid == 0) {
+                    sel = select_top<D>(rsc, ncr);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
-                            if (c < ncr) cidx[c] = sel_at(sel, c);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        int slot = -1;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            if (c < ncr && sel_at(sel, c) == row0 + i) slot = c;
-                        if (slot >= 0) {
-                            float *dst = w.comp_row_vec + ((size_t)u * ncr + slot) * D + col0;
-                            if constexpr (CL == 4)
-                                *reinterpret_cast<float4 *>(dst) =
-                                    make_float4(acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y);
-                            else
-                                *reinterpret_cast<float2 *>(dst) = acc[i][0];
-#pragma unroll
-                            for (int m = 0; m < CL / 2; ++m) acc[i][m] = make_float2(0.0f, 0.0f);
-                        }
-                    }
+                            if (c < ncr && sel_at(sel, c) == row0 + i) rslot[i] = c;
                 }
 
-                // 2b, 3. column statistics of the row-zeroed residual: partials over this
-                // CTA's rows, sent to every CTA, reduced in rank order
+                // 2b, 3. column statistics of the row-zeroed residual (the chosen rows
+                // count as zero): partials over this CTA's rows, sent to every CTA,
+                // reduced in rank order
 #pragma unroll
                 for (int c = 0; c < CL; ++c) {
                     float sq = 0.0f, mx = 0.0f;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const float x = fabsf(at(i, c));
+                        const float x = rslot[i] >= 0 ? 0.0f : fabsf(at(i, c));
                         sq = sq + x * x;
                         mx = fmaxf(mx, x);
                     }
@@ -393,8 +381,23 @@ __global__ void __launch_bounds__(kThreads) flush_split_kernel(EncodeArgs a) {
                 const uint2 csel = select_top<D>(sh_score, ncc);
                 if (rank == 0 && tid == 0) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
+                    for (int c = 0; c < 8; ++c) {
+                        if (c < ncr) cidx[c] = sel_at(sel, c);
                         if (c < ncc) cidx[ncr + c] = sel_at(csel, c);
+                    }
+                }
+                // the chosen rows: stored, then zeroed
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (rslot[i] >= 0) {
+                        float *dst = w.comp_row_vec + ((size_t)u * ncr + rslot[i]) * D + col0;
+                        if constexpr (CL == 4)
+                            *reinterpret_cast<float4 *>(dst) = make_float4(acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y);
+                        else
+                            *reinterpret_cast<float2 *>(dst) = acc[i][0];
+#pragma unroll
+                        for (int m = 0; m < CL / 2; ++m) acc[i][m] = make_float2(0.0f, 0.0f);
+                    }
                 }
                 if (tid < D) {
                     bool chosen = false;
@@ -467,7 +470,9 @@ __global__ void __launch_bounds__(kThreads) flush_split_kernel(EncodeArgs a) {
         }
         __syncthreads();                                 // before the counts are read again
     }
-    cluster.sync();   // no CTA leaves while another may still write its shared memory
+    // No CTA leaves while another may still write its shared memory; nothing is
+    // exchanged here, so the arrival orders no memory.
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
 template <int D, bool KDA, typename KeyT>

@@ -9,7 +9,10 @@ and, with --flush, one window flush.  Launch order: the prefill's encode
 launch (windowed/naive modes), then the T decode launches, then the flush.
 With --prompt P the state is instead prefilled from a P-token prompt by one
 token-prefill launch (lq_prefill_tokens).  --batch overrides the workload's
-batch (smaller captures).
+batch (smaller captures).  With --ragged-due S the handle is ragged: W - 1
+decode launches with every sequence active, one with only the first S
+sequences active (their windows are then full), then one flush of the due
+units (the cluster flush); --tokens and --flush are ignored.
 """
 from __future__ import annotations
 
@@ -28,6 +31,7 @@ def main() -> None:
     ap.add_argument("--flush", action="store_true")
     ap.add_argument("--prompt", type=int, default=0)
     ap.add_argument("--batch", type=int, default=0)
+    ap.add_argument("--ragged-due", type=int, default=-1)
     args = ap.parse_args()
     wl = inputs.WORKLOADS[args.workload]
     if args.batch:
@@ -40,9 +44,14 @@ def main() -> None:
     tb = inputs.tokens_on_device(wl.seed, T, wl.batch, wl.heads, wl.d_k, wl.d_v, wl.per_channel_gate, wl.dtype, dev)
     S0 = 0.3 * torch.randn(wl.batch, wl.heads, wl.d_v, wl.d_k, device=dev,
                            generator=torch.Generator(device=dev).manual_seed(wl.seed))
+    ragged = args.ragged_due >= 0
+    if ragged:
+        T = wl.window
+        tb = inputs.tokens_on_device(wl.seed, T, wl.batch, wl.heads, wl.d_k, wl.d_v, wl.per_channel_gate, wl.dtype,
+                                     dev)
     st = lq.DecodeState(wl.batch, wl.heads, wl.d_k, window=wl.window, n_comp_rows=wl.n_comp_rows,
                         n_comp_cols=wl.n_comp_cols, gate="channel" if wl.per_channel_gate else "scalar",
-                        mode=args.mode, in_dtype=wl.dtype, device=dev)
+                        mode=args.mode, in_dtype=wl.dtype, ragged=ragged, device=dev)
     if args.prompt:
         pb = inputs.tokens_on_device(wl.seed + 1, args.prompt, wl.batch, wl.heads, wl.d_k, wl.d_v,
                                      wl.per_channel_gate, wl.dtype, dev)
@@ -51,15 +60,23 @@ def main() -> None:
     else:
         st.prefill(S0)
     out = torch.empty(wl.batch, wl.heads, wl.d_v, dtype=torch.float32, device=dev)
-    for t in range(T):
-        st.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=out)
-    if args.flush:
+    if ragged:
+        act = torch.ones(wl.batch, dtype=torch.uint8, device=dev)
+        for t in range(T):
+            if t == T - 1:
+                act[args.ragged_due:] = 0
+            st.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=out, active=act)
         st.flush()
+    else:
+        for t in range(T):
+            st.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=out)
+        if args.flush:
+            st.flush()
     status = st.device_status()
     if status != lq.LQ_OK:
         raise lq.LQError(status, "profile_case")
     print(f"profile_case: {wl.name} batch={wl.batch} mode={args.mode} prompt={args.prompt} tokens={T} "
-          f"flush={args.flush} ok")
+          f"flush={args.flush} ragged_due={args.ragged_due} ok")
 
 
 if __name__ == "__main__":
