@@ -160,3 +160,20 @@ def test_full_size_prompt_sampled_units():
     o_gpu = out.reshape(T, B * H, d)[:, units].cpu().double().numpy().transpose(1, 0, 2)
     assert rel_l2(S_gpu, r.S_final) <= 1e-5
     assert rel_l2(o_gpu, r.o) <= 1e-5
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_naive_mode_codec_on_the_final_state(d):
+    """Naive per-token INT8 handles encode the prompt's final state with their
+    own codec (no compensators, no smoothing), bit for bit."""
+    B, H, T = 2, 3, 19
+    tb, S0 = _prompt(d, "scalar", torch.bfloat16, B, H, T, seed=29 + d)
+    ref, _ = _gpu_prefill("fp32", d, "scalar", torch.bfloat16, tb, S0, outputs=False)
+    st, _ = _gpu_prefill("naive", d, "scalar", torch.bfloat16, tb, S0, outputs=False)
+    S = ref.view("state_f32").cpu()
+    p = oracle_params(d, nr=0, nc=0, smooth=0, mode="naive")
+    for u in range(B * H):
+        b, h = divmod(u, H)
+        e = oracle.encode(p, S[b, h].double().numpy())
+        np.testing.assert_array_equal(st.view("codes")[b, h].cpu().numpy(), e.Q)
+        np.testing.assert_array_equal(st.view("row_scale")[b, h].cpu().numpy(), e.sigma)
