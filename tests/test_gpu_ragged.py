@@ -270,3 +270,97 @@ def test_ragged_restart_from_prompts_of_different_lengths(gate):
     assert rel_l2(np.concatenate(pgot), np.concatenate(pref)) <= 1e-5
     err = rel_l2(np.concatenate(got), np.concatenate(ref))
     assert err <= 1e-3, err
+
+
+@pytest.mark.parametrize("seed", [101, 202])
+def test_ragged_random_operation_mix(seed):
+    """Random masked decodes with a flush after each step, interleaved with
+    sequence restarts from a state or from a prompt and with pending flushes.
+    Each unit's outputs follow the oracle over its own segments: a restart
+    starts a segment from its new state (after the prompt's FP32 recurrence);
+    a pending flush ends the unit's partial window, so its next segment starts
+    from the oracle's state at that token."""
+    d, B, H, W, T, P = 64, 4, 2, 5, 36, 6
+    rng = np.random.default_rng(seed)
+    tb = inputs.tokens(seed, 0, T, B, H, d, d, False)
+    pb = inputs.tokens(seed + 1, 0, P, B, H, d, d, False)
+    gen = torch.Generator().manual_seed(seed)
+    S0 = 0.5 * torch.randn(B, H, d, d, generator=gen)
+    S1 = 0.5 * torch.randn(B, H, d, d, generator=gen)
+    st = lq.DecodeState(B, H, d, window=W, n_comp_rows=1, n_comp_cols=1, ragged=True, device=DEV)
+    st.prefill(S0.to(DEV).contiguous())
+    tbd, pbd = to_device(tb, DEV), to_device(pb, DEV)
+    out = torch.full((T, B, H, d), float("nan"), device=DEV)
+    pout = torch.full((P, B, H, d), float("nan"), device=DEV)
+    # per sequence: a list of segments (kind, start info, token steps)
+    segs = [[["state", "S0", []]] for _ in range(B)]
+    fill = np.zeros(B, dtype=np.int64)
+    prompt_used = False
+    events = {"state": 0, "prompt": 0, "pending": 0}
+    for t in range(T):
+        event = rng.random()
+        if event < 0.08 and t > 0:                                   # restart sequences from a state
+            mask = (rng.random(B) < 0.5).astype(np.uint8)
+            st.prefill_sequences(S1.to(DEV).contiguous(), torch.tensor(mask, device=DEV))
+            events["state"] += 1
+            for b in np.nonzero(mask)[0]:
+                segs[b].append(["state", "S1", []])
+                fill[b] = 0
+        elif event < 0.14 and t > 0 and not prompt_used:            # restart from prompts
+            mask = (rng.random(B) < 0.5).astype(np.uint8)
+            lengths = rng.integers(0, P + 1, B).astype(np.int32)
+            st.prefill_sequences_tokens(pbd.q, pbd.k, pbd.v, pbd.g, pbd.beta, torch.tensor(mask, device=DEV),
+                                        torch.tensor(lengths, device=DEV), S0=S1.to(DEV).contiguous(), out=pout)
+            prompt_used = True
+            events["prompt"] += 1
+            for b in np.nonzero(mask)[0]:
+                segs[b].append(["prompt", int(lengths[b]), []])
+                fill[b] = 0
+        elif event < 0.2 and t > 0:                                  # end every partial window
+            st.flush_pending()
+            events["pending"] += 1
+            for b in range(B):
+                if fill[b] > 0:
+                    segs[b].append(["continue", None, []])
+                fill[b] = 0
+        act = rng.random(B) < 0.7
+        st.decode_step(tbd.q[t], tbd.k[t], tbd.v[t], tbd.g[t], tbd.beta[t], out=out[t],
+                       active=torch.tensor(act.astype(np.uint8), device=DEV))
+        st.flush()
+        for b in np.nonzero(act)[0]:
+            segs[b][-1][2].append(t)
+            fill[b] = (fill[b] + 1) % W
+    assert min(events.values()) >= 1, events          # the seed exercises every operation
+    assert st.device_status() == lq.LQ_OK, lq.last_error()
+    assert (st.fills().cpu().numpy() == fill[:, None]).all()
+    o_gpu, p_gpu = out.cpu().numpy(), pout.cpu().numpy()
+    pw = oracle_params(d, W, 1, 1, "scalar", "window")
+    pf = oracle_params(d, W, 1, 1, "scalar", "fp32")
+    q, k, v, g, beta = unit_inputs(tb, range(B * H))
+    pq, pk, pv, pg, pbeta = unit_inputs(pb, range(B * H))
+    got, ref = [], []
+    for b in range(B):
+        for h in range(H):
+            u = b * H + h
+            S = None
+            for kind, info, steps in segs[b]:
+                if kind == "state":
+                    S = (S0 if info == "S0" else S1)[b, h].double().numpy()[None]
+                elif kind == "prompt":
+                    S = S1[b, h].double().numpy()[None]
+                    if info:
+                        rp = oracle.run(pf, S, pq[u:u + 1, :info], pk[u:u + 1, :info], pv[u:u + 1, :info],
+                                        pg[u:u + 1, :info], pbeta[u:u + 1, :info], snapshots=False)
+                        got.append(p_gpu[:info, b, h])
+                        ref.append(rp.o[0])
+                        S = rp.S_final
+                if not steps:
+                    continue
+                s = np.array(steps)
+                r = oracle.run(pw, S, q[u:u + 1, s], k[u:u + 1, s], v[u:u + 1, s], g[u:u + 1, s],
+                               beta[u:u + 1, s], snapshots=False)
+                got.append(o_gpu[s, b, h])
+                ref.append(r.o[0])
+                S = r.S_final                 # a later "continue" segment starts here
+    err = rel_l2(np.concatenate(got), np.concatenate(ref))
+    assert err <= 1e-3, err
