@@ -159,3 +159,25 @@ def test_prefill_tokens_validates_on_the_host():
     assert L.lq_prefill_tokens(h, odd, p, p, p, p, p, 4, None, None) == lq.LQ_ERR_INVALID_ARG     # S0: 16 B
     assert L.lq_prefill_tokens(None, None, p, p, p, p, p, 4, None, None) == lq.LQ_ERR_INVALID_ARG
     assert L.lq_state_destroy(h) == lq.LQ_OK
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without liblq.so the binding raises; there is no fallback path."""
+    import subprocess
+    import sys
+    code = (
+        "import sys, torch\n"
+        "from recurrent_state_quantization_lq_b200 import lq\n"
+        f"lq.LIB_PATH = {str(tmp_path / 'absent' / 'liblq.so')!r}\n"
+        "try:\n"
+        "    lq.workspace_bytes(lq.make_config(1, 1, 64))\n"
+        "except RuntimeError as e:\n"
+        "    print('raised', 'missing' in str(e))\n"
+        "    sys.exit(0)\n"
+        "sys.exit(3)\n"
+    )
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "raised True" in r.stdout
