@@ -41,6 +41,8 @@
  *    device (a gate sum out of the safe range, a bounded wait that expired)
  *    are recorded in the workspace's error word and reported by
  *    lq_device_status().  No kernel traps or asserts.
+ *  - Tracing.  Every call that enqueues device work opens an NVTX range named
+ *    after the call, so timeline tools group its kernels under it.
  *  - Window phase.  By default all sequences of a handle share one window
  *    phase: the handle counts buffered tokens (lq_window_fill) on the host.
  *    A ragged handle (cfg.ragged = 1, windowed mode) keeps one count per
@@ -263,6 +265,21 @@ LQ_API lq_status lq_prefill_sequences_tokens(lq_handle h, const float *d_S0, con
                                              const void *d_v, const float *d_g, const float *d_beta,
                                              int32_t max_tokens, const int32_t *d_lengths, const uint8_t *d_mask,
                                              float *d_o, void *stream);
+
+/*
+ * Resume from a checkpoint.  A handle's whole state is its workspace plus, for
+ * a shared-phase handle, the host count lq_window_fill().  To checkpoint: call
+ * lq_device_status() (it synchronizes the stream), then copy the workspace's
+ * lq_workspace_bytes() bytes and note lq_window_fill().  To resume: create a
+ * handle with the same lq_config over a workspace holding those bytes (the
+ * copy may sit at another address or on another device), then call this with
+ * the noted count.  n_buf: tokens buffered in the shared window, 0..W
+ * (windowed mode), 0 in the other modes; a ragged handle takes its counts
+ * from the workspace and ignores n_buf (pass 0).  No device work; the next
+ * decode, flush or prefill continues exactly where the checkpoint stood.
+ * Errors: LQ_ERR_INVALID_ARG for a bad handle or an n_buf out of range.
+ */
+LQ_API lq_status lq_state_resume(lq_handle h, int32_t n_buf);
 
 /* Tokens buffered in the current window (0..W); -1 for a bad or ragged handle
  * (a ragged handle's counts are on the device, at lq_layout.fill). */

@@ -8,6 +8,8 @@
 #include <string>
 
 #include "lq.h"
+#include <nvtx3/nvToolsExt.h>
+
 #include "lq_kernels.h"
 
 namespace {
@@ -122,6 +124,15 @@ namespace {
 
 bool check_handle(lq_handle h) { return h != nullptr && h->magic == kMagic; }
 
+// An NVTX range around a stream-ordered call, for timeline tools (nsys, ncu);
+// nearly free when no tool is attached.
+struct Range {
+    explicit Range(const char *name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range &) = delete;
+    Range &operator=(const Range &) = delete;
+};
+
 lq::Views views(lq_handle h) {
     lq::Views v;
     unsigned char *b = h->ws;
@@ -203,12 +214,24 @@ lq_status lq_state_destroy(lq_handle h) {
     return LQ_OK;
 }
 
+lq_status lq_state_resume(lq_handle h, int32_t n_buf) {
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    const lq_config &c = h->cfg;
+    const int32_t max_buf = (c.mode == LQ_MODE_WINDOW && !c.ragged) ? c.window : 0;
+    if (n_buf < 0 || n_buf > max_buf) return fail(LQ_ERR_INVALID_ARG, "n_buf out of range for this handle");
+    h->n_buf = n_buf;
+    h->prefilled = 1;
+    h->aligned = 0;                      // ragged: the phases are whatever the counts say
+    return LQ_OK;
+}
+
 int32_t lq_window_fill(lq_handle h) {
     if (!check_handle(h) || h->cfg.ragged) return -1;   // ragged counts live on the device
     return h->n_buf;
 }
 
 lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream) {
+    Range nvtx_range("lq_prefill_state");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
     if (d_S0 != nullptr && !aligned(d_S0, 16)) return fail(LQ_ERR_INVALID_ARG, "S0 must be 16-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -251,6 +274,7 @@ lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream) {
 
 lq_status lq_prefill_tokens(lq_handle h, const float *d_S0, const void *d_q, const void *d_k, const void *d_v,
                             const float *d_g, const float *d_beta, int32_t n_tokens, float *d_o, void *stream) {
+    Range nvtx_range("lq_prefill_tokens");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
     if (n_tokens < 0) return fail(LQ_ERR_INVALID_ARG, "negative n_tokens");
     if (n_tokens == 0) return lq_prefill_state(h, d_S0, stream);
@@ -295,6 +319,7 @@ lq_status lq_prefill_tokens(lq_handle h, const float *d_S0, const void *d_q, con
 lq_status lq_prefill_sequences_tokens(lq_handle h, const float *d_S0, const void *d_q, const void *d_k,
                                       const void *d_v, const float *d_g, const float *d_beta, int32_t max_tokens,
                                       const int32_t *d_lengths, const uint8_t *d_mask, float *d_o, void *stream) {
+    Range nvtx_range("lq_prefill_sequences_tokens");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
     const lq_config &c = h->cfg;
     if (!c.ragged) return fail(LQ_ERR_STATE, "lq_prefill_sequences_tokens needs a ragged handle");
@@ -410,28 +435,33 @@ lq_status flush_impl(lq_handle h, int flush_min, void *stream) {
 
 lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, const void *d_v, const float *d_g,
                          const float *d_beta, float *d_o, void *stream) {
+    Range nvtx_range("lq_decode_step");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
     return decode_impl(h, d_q, d_k, d_v, d_g, d_beta, nullptr, d_o, stream);
 }
 
 lq_status lq_decode_step_active(lq_handle h, const void *d_q, const void *d_k, const void *d_v, const float *d_g,
                                 const float *d_beta, const uint8_t *d_active, float *d_o, void *stream) {
+    Range nvtx_range("lq_decode_step_active");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
     if (!h->cfg.ragged) return fail(LQ_ERR_STATE, "lq_decode_step_active needs a ragged handle");
     return decode_impl(h, d_q, d_k, d_v, d_g, d_beta, d_active, d_o, stream);
 }
 
 lq_status lq_window_flush(lq_handle h, void *stream) {
+    Range nvtx_range("lq_window_flush");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
     return flush_impl(h, h->cfg.window, stream);
 }
 
 lq_status lq_window_flush_pending(lq_handle h, void *stream) {
+    Range nvtx_range("lq_window_flush_pending");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
     return flush_impl(h, 1, stream);
 }
 
 lq_status lq_prefill_sequences(lq_handle h, const float *d_S0, const uint8_t *d_mask, void *stream) {
+    Range nvtx_range("lq_prefill_sequences");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
     const lq_config &c = h->cfg;
     if (!c.ragged) return fail(LQ_ERR_STATE, "lq_prefill_sequences needs a ragged handle");
@@ -458,6 +488,7 @@ lq_status lq_prefill_sequences(lq_handle h, const float *d_S0, const uint8_t *d_
 }
 
 lq_status lq_device_status(lq_handle h, void *stream) {
+    Range nvtx_range("lq_device_status");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaStreamSynchronize(s);

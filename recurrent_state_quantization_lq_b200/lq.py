@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.lq_prefill_tokens.restype = i32
         L.lq_prefill_sequences_tokens.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
         L.lq_prefill_sequences_tokens.restype = i32
+        L.lq_state_resume.argtypes = [vp, i32]
+        L.lq_state_resume.restype = i32
         L.lq_window_fill.argtypes = [vp]
         L.lq_window_fill.restype = i32
         L.lq_device_status.argtypes = [vp, vp]
@@ -262,6 +264,21 @@ class DecodeState:
                                                       _stream_ptr(stream, self.device)),
                     "lq_prefill_sequences_tokens")
         return out
+
+    def checkpoint(self, stream=None) -> tuple[torch.Tensor, int]:
+        """A copy of the whole state: the workspace bytes and the shared-window
+        count (0 on a ragged state, whose counts are in the workspace)."""
+        status = self.device_status(stream)
+        if status != LQ_OK:
+            raise LQError(status, "checkpoint of a state with a device error")
+        return self.workspace.clone(), max(self.fill, 0)
+
+    def resume(self, workspace: torch.Tensor, n_buf: int) -> None:
+        """Continue from a checkpoint() of a state with the same configuration."""
+        assert workspace.dtype == torch.uint8 and workspace.numel() == self.workspace.numel()
+        self.workspace.copy_(workspace)
+        torch.cuda.synchronize(self.device)
+        self._check(lib().lq_state_resume(self._h, int(n_buf)), "lq_state_resume")
 
     @property
     def fill(self) -> int:

@@ -14,7 +14,7 @@ def test_exports_every_declared_symbol():
                           "lq_prefill_state", "lq_decode_step", "lq_window_flush", "lq_window_fill",
                           "lq_device_status", "lq_state_destroy", "lq_last_error_string",
                           "lq_decode_step_active", "lq_window_flush_pending", "lq_prefill_sequences",
-                          "lq_prefill_tokens", "lq_prefill_sequences_tokens"}
+                          "lq_prefill_tokens", "lq_prefill_sequences_tokens", "lq_state_resume"}
     L = lq.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -181,3 +181,24 @@ def test_missing_library_fails_loudly(tmp_path):
     r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "raised True" in r.stdout
+
+
+def test_resume_validates_on_the_host():
+    L = lq.lib()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: resume does no device work
+    for kw, ok, bad in (({"window": 8}, (0, 5, 8), (-1, 9)),
+                        ({"window": 8, "mode": "naive"}, (0,), (1,)),
+                        ({"window": 8, "mode": "fp32"}, (0,), (1,)),
+                        ({"window": 8, "ragged": True}, (0,), (1,))):
+        cfg = lq.make_config(2, 3, 64, **kw)
+        h = ctypes.c_void_p()
+        assert L.lq_state_create(ctypes.byref(cfg), fake, lq.workspace_bytes(cfg), ctypes.byref(h)) == lq.LQ_OK
+        for n in ok:
+            assert L.lq_state_resume(h, n) == lq.LQ_OK, (kw, n)
+        for n in bad:
+            assert L.lq_state_resume(h, n) == lq.LQ_ERR_INVALID_ARG, (kw, n)
+        if not kw.get("ragged") and kw.get("mode", "window") == "window":
+            L.lq_state_resume(h, 5)
+            assert L.lq_window_fill(h) == 5
+        assert L.lq_state_destroy(h) == lq.LQ_OK
+    assert L.lq_state_resume(None, 0) == lq.LQ_ERR_INVALID_ARG
