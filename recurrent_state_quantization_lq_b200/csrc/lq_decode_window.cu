@@ -25,7 +25,8 @@
 // slot has a full mbarrier (bytes landed) and an empty mbarrier that every
 // consumer thread arrives on after its last read, so no block-wide barrier is
 // spent on releasing slots; the consumers meet at one barrier after the
-// operand prep and one per chunk.
+// operand prep and one per chunk.  Each thread keeps its row scale sigma_i in a
+// register, so the meta slot goes back before the INT8 pass starts.
 //
 // The INT8 pass is an exact integer dot product on the tensor cores.  Each
 // 32-column block of y^q = s*x^q and y^k = s*x^k is written as
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const int meta_slot = slot;
         advance();
         double G_j = 0.0;
-        float key_out = 0.0f, v_i = 0.0f;
+        float key_out = 0.0f, v_i = 0.0f, sig_i = 0.0f;
         if (owns_row) {
             const int j = tid;
             float gam;
@@ -382,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const float kj = to_f32(reinterpret_cast<const InT *>(mp + M.kin)[j]);
             const float sj = reinterpret_cast<const float *>(mp + M.s)[j];
             v_i = to_f32(reinterpret_cast<const InT *>(mp + M.vin)[j]);
+            sig_i = reinterpret_cast<const float *>(mp + M.sig)[j];
             const float xq = gam * qj, xk = gam * kj;
             sXq[j] = xq;
             sXk[j] = xk;
@@ -492,14 +494,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 }
             }
         }
+        // this thread's last read of the meta segment: the slot goes back to the
+        // producer before the INT8 pass, so the next copy starts that much earlier
+        mbar_arrive(&empty[meta_slot]);
 
         // ---------------------------- A2: one pass over the INT8 tile
-        // a_i = sigma_i sum_j Q_ij y^q_j and b_i = sigma_i sum_j Q_ij y^k_j, as
+        // sum_j Q_ij y^q_j and sum_j Q_ij y^k_j (sigma_i is applied at emit), as
         // exact int8 products on the tensor cores (see the file comment)
         bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
         {
             const unsigned char *tile = ring + slot * kSlotBytes;
-            const float *sSig = reinterpret_cast<const float *>(mp + M.sig);
             const int g = lane >> 2, c4 = lane & 3;
             uint32_t bf[KBLK][2];                  // B fragments: digit column g, k = 4*c4 (+16)
 #pragma unroll
@@ -536,12 +540,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
                 if ((c4 & 1) == 0) {
                     float *dst = (c4 == 0) ? sA : sB;
-                    dst[m0 + g] = sSig[m0 + g] * v0;
-                    dst[m0 + g + 8] = sSig[m0 + g + 8] * v1;
+                    dst[m0 + g] = v0;
+                    dst[m0 + g + 8] = v1;
                 }
             }
         }
-        mbar_arrive(&empty[meta_slot]);            // done with the meta segment (row scales last)
         mbar_arrive(&empty[slot]);                 // done with the INT8 tile
         advance();
 
@@ -610,7 +613,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // ------------------------------------------------ A4: emit and append
         if (owns_row) {
             const int i = tid;
-            const float sk = acc.x + sB[i], so = acc.y + sA[i];
+            // sigma_i times the INT8 products, rounded before the sum as a product of its own
+            const float sk = acc.x + __fmul_rn(sig_i, sB[i]), so = acc.y + __fmul_rn(sig_i, sA[i]);
             const float delta = beta * (v_i - sk);
             const size_t slot_g = (size_t)u * w.window + n_buf;
             a.o[(size_t)u * D + i] = fmaf(delta, kq, so);
