@@ -164,6 +164,14 @@ def test_window_decode_variants(d, gate, W, nr, nc):
     _window_case(d, gate, torch.bfloat16, W, nr, nc, B, H, T, seed=11 + W, S0_kind="normal")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_window_decode_fp32_inputs(d, gate):
+    """FP32 q, k, v (so FP32 buffered keys): every decode instantiation with FP32 inputs."""
+    W = 37
+    _window_case(d, gate, torch.float32, W, 2, 2, 2, 3, 2 * W + 5, seed=71, S0_kind="normal")
+
+
 def test_window_decode_planted_outliers_maxabs_nosmooth():
     d, B, H, W = 128, 2, 4, 16
     for smooth, select in ((0, "l2"), (1, "maxabs")):

@@ -88,7 +88,8 @@ def _ragged_case(d, gate, dtype, W, nr, nc, B, H, T, seed, join_at=None, p_activ
 
 @pytest.mark.parametrize("d,gate,dtype", [(64, "scalar", torch.bfloat16), (128, "scalar", torch.bfloat16),
                                           (128, "channel", torch.bfloat16), (64, "scalar", torch.float32),
-                                          (64, "channel", torch.bfloat16), (128, "scalar", torch.float32)])
+                                          (64, "channel", torch.bfloat16), (128, "scalar", torch.float32),
+                                          (128, "channel", torch.float32), (64, "channel", torch.float32)])
 def test_ragged_phases_match_per_sequence_oracle(d, gate, dtype):
     _ragged_case(d, gate, dtype, W=8, nr=2, nc=2, B=3, H=2, T=40, seed=31)
 
