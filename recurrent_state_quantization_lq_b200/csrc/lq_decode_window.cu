@@ -469,23 +469,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         for (int i = 0; i < D / 32; ++i) kq += sRed[i * Sh::RED];
         float2 acc = make_float2(0.0f, 0.0f);      // (S_{t-1} x^k, S_{t-1} x^q) parts of this row
         if (owns_row && ncomp > 0) {
-            // all index and vector loads first, then the dependent x loads
             const int32_t *cidx = reinterpret_cast<const int32_t *>(mp + M.cidx);
             const float *ccol = reinterpret_cast<const float *>(mp + M.ccol);
-            int jc[8], rc = -1;
-            float vcol[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const bool on = c < ncc;
-                jc[c] = on ? (cidx[ncr + c] & (D - 1)) : 0;   // in range whatever the workspace holds
-                vcol[c] = on ? ccol[c * D + tid] : 0.0f;
-                if (c < ncr && cidx[c] == tid) rc = c;
+            // column compensators, in order: (C x)_i = sum_c v_c[i] x_{j_c}
+#pragma unroll 2
+            for (int c = 0; c < ncc; ++c) {
+                const int jc = cidx[ncr + c] & (D - 1);      // in range whatever the workspace holds
+                const float vc = ccol[c * D + tid];
+                acc.x = fmaf(vc, sXk[jc], acc.x);
+                acc.y = fmaf(vc, sXq[jc], acc.y);
             }
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                acc.x = fmaf(vcol[c], sXk[jc[c]], acc.x);
-                acc.y = fmaf(vcol[c], sXq[jc[c]], acc.y);
-            }
+            int rc = -1;                           // this row's slot among the row compensators
+            for (int c = 0; c < ncr; ++c)
+                if (cidx[c] == tid) rc = c;
             if (rc >= 0) {
 #pragma unroll
                 for (int i = 0; i < D / 32; ++i) {
@@ -626,11 +622,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 reinterpret_cast<KeyT *>(w.buf_key)[slot_g * D + i] = static_cast<KeyT>(key_out);
             }
         }
-        if (!KDA && tid == 0) {
+        // one-thread bookkeeping on lanes of different warps, so that no warp
+        // carries all of it into the next unit's barrier
+        if (!KDA && tid == 32) {
             w.buf_gate[(size_t)u * w.window_pad + n_buf] = exp_of_double(-Gs);
             w.gate_sum[u] = Gs;
         }
-        if (RAGGED && tid == 0) a.fill[u] = n_buf + 1;
+        if (RAGGED && tid == 64) a.fill[u] = n_buf + 1;
         if (!KDA && un < units) {                  // next unit's G_t and gamma_t, off its critical path
             G_n = G_n + (double)g_n;
             gam_n = exp_of_double(G_n);
