@@ -199,13 +199,18 @@ __device__ __forceinline__ float2 block_scale(float m) {
 }
 
 // The four base-2^7 int8 digits of y * 2^-E (|y 2^-E| < 64), packed low to high.
+// Every |r| here is at most 64, so adding 1.5 * 2^23 rounds r to an integer
+// (to nearest, ties to even, as rintf) with no conversion instruction: the
+// sum minus 1.5 * 2^23 is the digit as a float, and the sum's low byte is its
+// two's-complement byte.
 __device__ __forceinline__ uint32_t digits4(float y, float down) {
     float r = y * down;
     uint32_t out = 0;
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-        const float d = rintf(r);
-        out |= ((uint32_t)(int)d & 0xffu) << (8 * p);
+        const float t = __fadd_rn(r, 12582912.0f);
+        const float d = __fsub_rn(t, 12582912.0f);
+        out |= (__float_as_uint(t) & 0xffu) << (8 * p);
         r = (r - d) * 128.0f;
     }
     return out;
