@@ -32,9 +32,15 @@
 // 32-column block of y^q = s*x^q and y^k = s*x^k is written as
 // y = 2^E (d_0 + d_1 2^-7 + d_2 2^-14 + d_3 2^-21) with int8 digits d_p and a
 // block exponent E (every step exact in FP32; the dropped remainder is below
-// 2^-27 of the block maximum).  mma.sync m16n8k32 s8 x s8 -> s32 then forms
-// Q d_p for all 8 (vector, digit) columns at once with exact int32 sums, and
-// the digits are recombined in FP32.  No per-byte widening is needed.
+// 2^-27 of the block maximum).  The products Q d_p of all 8 (vector, digit)
+// columns are exact int32 sums, and the digits are recombined in FP32; no
+// per-byte widening is needed.  For d = 128 one thread issues them on the
+// fifth-generation tensor cores (tcgen05.mma kind::i8: per 32-column block an
+// M = 128, N = 16, K = 32 product from the swizzled tile and the digit rows in
+// shared memory into tensor memory, lane i = row i) as soon as the tile has
+// landed, so the pass runs while the warps form the compensator terms; each
+// warp then reads its 32 rows back.  For d = 64 the warps use mma.sync
+// m16n8k32.  Both give the same sums and the same FP32 recombination.
 // Every wait is bounded; an expired wait records LQ_DEVERR_TIMEOUT and all
 // consumer warps leave together at their next barrier.
 #include <cuda.h>
@@ -67,14 +73,17 @@ struct Shape {
     static constexpr int C_GATE = C_KEY + KB * D * E;
     static constexpr int KBLK = D / 32;                            // 32-column blocks (one per prep warp)
     static constexpr int MT = D / 16 / kConsumerWarps;             // 16-row m-tiles per warp
+    // d = 128: the INT8 pass runs on tcgen05 (one thread issues it, the sums
+    // land in tensor memory, lane i = row i); d = 64: warp-level mma.sync
+    static constexpr bool TC = (D == 128);
     // consumer scratch, in floats: digits (8 x D int8), block scales, vectors,
     // products, coefficients (two buffers), compensator dots, reductions
     static constexpr int RED = 1 + 2 * 8;                          // kq, then (k, q) dots of 8 row comps
-    static constexpr int S_B8 = 0, S_EXP = 2 * D, S_XQ = S_EXP + 8, S_XK = S_XQ + D, S_QR = S_XK + D,
+    static constexpr int S_B8 = 0, S_EXP = S_B8 + (TC ? 4 * D : 2 * D), S_XQ = S_EXP + 8, S_XK = S_XQ + D, S_QR = S_XK + D,
                          S_KR = S_QR + D, S_A = S_KR + D, S_B = S_A + D, S_CF = S_B + D,
                          S_RED = S_CF + 64, S_FLOATS = S_RED + kConsumerWarps * RED;
     static constexpr int OFF_BARS = 4 * S_FLOATS;                  // then the ring, 1024-aligned
-    static constexpr int OFF_RING = align_up(OFF_BARS + 16 * kSlots, 1024);
+    static constexpr int OFF_RING = align_up(OFF_BARS + 16 * kSlots + 16, 1024);   // + MMA barrier, TMEM slot
     static constexpr int SMEM = OFF_RING + kSlots * kSlotBytes + 1024;   // + alignment slack
     static_assert(E >= 4 && E <= kPer * kConsumerWarps, "chunk size");
     static_assert(MT >= 1, "m-tiles");
@@ -184,6 +193,29 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
 
 // Exact int -> float for |x| < 2^22 without the conversion unit: at 1.5 * 2^23
 // the float spacing is 1, so the word 0x4B400000 + x is the number 1.5 * 2^23 + x.
+// tcgen05 pieces of the d = 128 INT8 pass.  Both operands are K-major with
+// 128-byte swizzle: rows of 128 int8 (one row of the state tile, or one digit
+// column), 8-row groups 1024 B apart, 16-byte pieces permuted by the row's
+// index mod 8 -- the layout the tile's 2-D tensor copy writes.
+constexpr int kTmemCols = 64;                 // 4 blocks x 16 accumulator columns
+// s32 accumulator, s8 A and B, both K-major, N = 16, M = 128
+constexpr uint32_t kI8Idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3fff);   // start address
+    d |= (uint64_t)(16 >> 4) << 16;           // leading byte offset (unused with this swizzle)
+    d |= (uint64_t)(1024 >> 4) << 32;         // stride byte offset: 8-row groups
+    d |= (uint64_t)1 << 46;                   // descriptor version
+    d |= (uint64_t)2 << 61;                   // 128-byte swizzle
+    return d;
+}
+__device__ __forceinline__ int sw128_off(int row, int kbyte) {
+    return (row >> 3) * 1024 + (row & 7) * 128 + ((((kbyte >> 4) ^ (row & 7))) << 4) + (kbyte & 15);
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
 __device__ __forceinline__ float i2f_exact(int x) { return __int_as_float(0x4B400000 + x) - 12582912.0f; }
 
 // 2^k as a float, for |k| <= 126.
@@ -237,16 +269,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     float *scr = reinterpret_cast<float *>(sm);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + Sh::OFF_BARS);
     uint64_t *empty = full + kSlots;
+    uint64_t *mma_bar = empty + kSlots;            // tcgen05 pass complete (d = 128)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 1);
     unsigned char *ring = sm + Sh::OFF_RING;
+    unsigned char *dig = sm + Sh::S_B8 * 4;        // digit operand (scratch starts at sm)
 
     if (tid == 0) {
         for (int i = 0; i < kSlots; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], kConsumers);
         }
+        mbar_init(mma_bar, 1);
         fence_mbar_init();
     }
+    if constexpr (Sh::TC) {
+        // the digit operand has 16 rows for N = 16; rows 8..15 stay zero
+        for (int i = tid; i < 1024 / 4; i += kThreads) reinterpret_cast<uint32_t *>(dig + 1024)[i] = 0u;
+        if (warp == 0) {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                         "r"(kTmemCols));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        }
+        tc_fence_before();
+    }
     __syncthreads();
+    if constexpr (Sh::TC) tc_fence_after();
 
     // ================================================================ producer
     if (warp == kConsumerWarps) {
@@ -331,6 +378,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     auto advance = [&]() {
         if (++slot == kSlots) { slot = 0; ph ^= 1u; }
     };
+    const uint32_t tmem = Sh::TC ? *tmem_slot : 0u;   // lane i = state row i
+    uint32_t mph = 0;                                 // phase of the tcgen05 pass barrier
     int u = blockIdx.x;
     float beta_n = 0.0f, g_n = 0.0f, gam_n = 0.0f;
     double G_n = 0.0;
@@ -402,8 +451,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const uint32_t dq = digits4(yq, eq.x), dk = digits4(yk, ek.x);
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
-                sB8[p * D + j] = (int8_t)((dq >> (8 * p)) & 0xff);
-                sB8[(4 + p) * D + j] = (int8_t)((dk >> (8 * p)) & 0xff);
+                if constexpr (Sh::TC) {            // digit column n is operand row n
+                    dig[sw128_off(p, j)] = (unsigned char)((dq >> (8 * p)) & 0xff);
+                    dig[sw128_off(4 + p, j)] = (unsigned char)((dk >> (8 * p)) & 0xff);
+                } else {
+                    sB8[p * D + j] = (int8_t)((dq >> (8 * p)) & 0xff);
+                    sB8[(4 + p) * D + j] = (int8_t)((dk >> (8 * p)) & 0xff);
+                }
             }
             if (lane == 0) {
                 sExp[warp] = eq.y;
@@ -463,9 +517,34 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
         }
         if (!KDA && tid == 0 && fabs(Gs) > kMaxAbsGateSum) report_error(w.err, LQ_DEVERR_RANGE, u, -1);
+        if constexpr (Sh::TC) {
+            fence_proxy_async_smem();              // the digits are read by the tensor cores
+            tc_fence_before();                     // this thread's last tensor-memory loads come first
+        }
         if (consumer_sync_or(bad)) {
             if (tid == 0) report_error(w.err, LQ_DEVERR_TIMEOUT, u, 0);
-            return;
+            goto consumers_done;
+        }
+
+        if constexpr (Sh::TC) {
+            // One thread starts the INT8 pass as soon as the tile is in: per
+            // 32-column block kb an M = 128, N = 16, K = 32 s8 product into
+            // tensor-memory columns 16 kb ..  It runs under the compensator terms.
+            if (tid == 0) {
+                bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
+                if (bad) report_error(w.err, LQ_DEVERR_TIMEOUT, u, -4);
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(ring + slot * kSlotBytes), b0 = smem_u32(dig);
+#pragma unroll
+                for (int kb = 0; kb < KBLK; ++kb) {
+                    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                                 "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+                                 ::"r"(tmem + (uint32_t)(16 * kb)), "l"(sw128_desc(a0 + 32 * kb)),
+                                 "l"(sw128_desc(b0 + 32 * kb)), "r"(kI8Idesc), "r"(0));
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                             ::"r"(smem_u32(mma_bar)) : "memory");
+            }
         }
 
         // kq, this row's compensator contributions (row and column ones)
@@ -502,8 +581,35 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // ---------------------------- A2: one pass over the INT8 tile
         // sum_j Q_ij y^q_j and sum_j Q_ij y^k_j (sigma_i is applied at emit), as
         // exact int8 products on the tensor cores (see the file comment)
-        bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
-        {
+        // (with the tensor-core pass, thread 0 waited for the tile; its completion
+        // tells every thread the tile is in and read)
+        if constexpr (!Sh::TC) bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
+        float p8q = 0.0f, p8k = 0.0f;              // TC: this thread's row of the two products
+        if constexpr (Sh::TC) {
+            bad |= !mbar_wait(mma_bar, mph, kWaitBudgetCycles);
+            mph ^= 1u;
+            tc_fence_after();
+            __syncwarp();
+            // digit columns 0..3 belong to y^q, 4..7 to y^k; the digits combine in
+            // the order the warp-level pass uses (digits 0, 1 and 2, 3 in two sums)
+            float s01q = 0.0f, s23q = 0.0f, s01k = 0.0f, s23k = 0.0f;
+#pragma unroll
+            for (int kb = 0; kb < KBLK; ++kb) {
+                uint32_t r[8];
+                asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                             : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                               "=r"(r[7])
+                             : "r"(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(16 * kb)));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                const float sq = sExp[kb], sk = sExp[4 + kb];
+                s01q = fmaf(sq, fmaf(i2f_exact((int)r[1]), 0x1p-7f, i2f_exact((int)r[0])), s01q);
+                s23q = fmaf(sq, fmaf(i2f_exact((int)r[3]), 0x1p-21f, i2f_exact((int)r[2]) * 0x1p-14f), s23q);
+                s01k = fmaf(sk, fmaf(i2f_exact((int)r[5]), 0x1p-7f, i2f_exact((int)r[4])), s01k);
+                s23k = fmaf(sk, fmaf(i2f_exact((int)r[7]), 0x1p-21f, i2f_exact((int)r[6]) * 0x1p-14f), s23k);
+            }
+            p8q = s01q + s23q;
+            p8k = s01k + s23k;
+        } else {
             const unsigned char *tile = ring + slot * kSlotBytes;
             const int g = lane >> 2, c4 = lane & 3;
             uint32_t bf[KBLK][2];                  // B fragments: digit column g, k = 4*c4 (+16)
@@ -589,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
             if (consumer_sync_or(bad)) {
                 if (tid == 0) report_error(w.err, LQ_DEVERR_TIMEOUT, u, 1 + c);
-                return;
+                goto consumers_done;
             }
             if (owns_row) {
                 float2 p[4] = {acc, make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
@@ -608,14 +714,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
         if (nchunks == 0 && consumer_sync_or(bad)) {
             if (tid == 0) report_error(w.err, LQ_DEVERR_TIMEOUT, u, 0);
-            return;
+            goto consumers_done;
         }
 
         // ------------------------------------------------ A4: emit and append
         if (owns_row) {
             const int i = tid;
             // sigma_i times the INT8 products, rounded before the sum as a product of its own
-            const float sk = acc.x + __fmul_rn(sig_i, sB[i]), so = acc.y + __fmul_rn(sig_i, sA[i]);
+            const float pk = Sh::TC ? p8k : sB[i], pq = Sh::TC ? p8q : sA[i];
+            const float sk = acc.x + __fmul_rn(sig_i, pk), so = acc.y + __fmul_rn(sig_i, pq);
             const float delta = beta * (v_i - sk);
             const size_t slot_g = (size_t)u * w.window + n_buf;
             a.o[(size_t)u * D + i] = fmaf(delta, kq, so);
@@ -638,6 +745,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             G_n = G_n + (double)g_n;
             gam_n = exp_of_double(G_n);
         }
+    }
+consumers_done:
+    // every consumer warp gets here (normal end, or a timeout all of them saw at
+    // the same barrier); no tensor-core pass is in flight, so the tensor memory
+    // goes back once all warps' loads are done
+    if constexpr (Sh::TC) {
+        tc_fence_before();
+        asm volatile("bar.sync %0, %1;" ::"r"(kConsumerBarrier), "r"(kConsumers) : "memory");
+        tc_fence_after();
+        if (warp == 0)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
 }
 
