@@ -63,7 +63,7 @@ constexpr double kMaxAbsGateSum = 80.0;
 
 __host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-template <int D, bool KDA, typename InT, typename KeyT>
+template <int D, bool KDA, typename InT, typename KeyT, bool TCP>
 struct Shape {
     static constexpr int KB = (int)sizeof(KeyT);
     static constexpr int ENTRY = 4 * D + KB * D + (KDA ? 0 : 4);   // bytes per buffered entry
@@ -73,9 +73,9 @@ struct Shape {
     static constexpr int C_GATE = C_KEY + KB * D * E;
     static constexpr int KBLK = D / 32;                            // 32-column blocks (one per prep warp)
     static constexpr int MT = D / 16 / kConsumerWarps;             // 16-row m-tiles per warp
-    // d = 128: the INT8 pass runs on tcgen05 (one thread issues it, the sums
-    // land in tensor memory, lane i = row i); d = 64: warp-level mma.sync
-    static constexpr bool TC = (D == 128);
+    // the INT8 pass on tcgen05 (one thread issues it, the sums land in tensor
+    // memory, lane i = row i; d = 128 only), else on warp-level mma.sync
+    static constexpr bool TC = TCP && (D == 128);
     // consumer scratch, in floats: digits (8 x D int8), block scales, vectors,
     // products, coefficients (two buffers), compensator dots, reductions
     static constexpr int RED = 1 + 2 * 8;                          // kq, then (k, q) dots of 8 row comps
@@ -247,10 +247,10 @@ __device__ __forceinline__ uint32_t digits4(float y, float down) {
     }
     return out;
 }
-template <int D, bool KDA, typename InT, typename KeyT, bool RAGGED>
+template <int D, bool KDA, typename InT, typename KeyT, bool RAGGED, bool TCP>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_window_kernel(DecodeArgs a, const __grid_constant__ CUtensorMap codes_map) {
-    using Sh = Shape<D, KDA, InT, KeyT>;
+    using Sh = Shape<D, KDA, InT, KeyT, TCP>;
     constexpr int E = Sh::E, KBLK = Sh::KBLK, MT = Sh::MT;
     const Views &w = a.w;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -772,12 +772,12 @@ int sm_count() {
     return cached[dev];
 }
 
-template <int D, bool KDA, typename InT, typename KeyT, bool RAGGED>
+template <int D, bool KDA, typename InT, typename KeyT, bool RAGGED, bool TCP>
 cudaError_t launch_r(const DecodeArgs &a, cudaStream_t s) {
-    using Sh = Shape<D, KDA, InT, KeyT>;
+    using Sh = Shape<D, KDA, InT, KeyT, TCP>;
     const Meta M = meta_layout<D, KDA, InT>(a.w.n_comp_rows, a.w.n_comp_cols, a.w.comp_index_stride);
     if (M.bytes > kSlotBytes || D * D > kSlotBytes) return cudaErrorInvalidValue;
-    auto kern = decode_window_kernel<D, KDA, InT, KeyT, RAGGED>;
+    auto kern = decode_window_kernel<D, KDA, InT, KeyT, RAGGED, TCP>;
     // The opt-in shared-memory size is set once per device, so that launches
     // inside a stream capture make no attribute calls.
     static bool opted_in[64] = {false};
@@ -795,9 +795,21 @@ cudaError_t launch_r(const DecodeArgs &a, cudaStream_t s) {
 }
 
 // Shared window phases compile without the per-unit counts and the active mask.
+// The tensor-core pass pays a tensor-memory allocation per CTA and a commit
+// round trip per unit; it is the faster one once the CTAs walk two units or
+// more each (measured: 1-5 % faster from 2048 units, up to 16 % slower at one
+// unit per CTA).  Both passes give the same sums.
+template <int D, bool KDA, typename InT, typename KeyT, bool RAGGED>
+cudaError_t launch_p(const DecodeArgs &a, cudaStream_t s) {
+    if constexpr (D == 128) {
+        if (a.w.units >= 2 * kCtasPerSm * sm_count()) return launch_r<D, KDA, InT, KeyT, RAGGED, true>(a, s);
+    }
+    return launch_r<D, KDA, InT, KeyT, RAGGED, false>(a, s);
+}
+
 template <int D, bool KDA, typename InT, typename KeyT>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
-    return a.fill != nullptr ? launch_r<D, KDA, InT, KeyT, true>(a, s) : launch_r<D, KDA, InT, KeyT, false>(a, s);
+    return a.fill != nullptr ? launch_p<D, KDA, InT, KeyT, true>(a, s) : launch_p<D, KDA, InT, KeyT, false>(a, s);
 }
 
 }  // namespace
