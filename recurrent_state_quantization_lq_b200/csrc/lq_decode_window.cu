@@ -34,13 +34,16 @@
 // block exponent E (every step exact in FP32; the dropped remainder is below
 // 2^-27 of the block maximum).  The products Q d_p of all 8 (vector, digit)
 // columns are exact int32 sums, and the digits are recombined in FP32; no
-// per-byte widening is needed.  For d = 128 one thread issues them on the
-// fifth-generation tensor cores (tcgen05.mma kind::i8: per 32-column block an
-// M = 128, N = 16, K = 32 product from the swizzled tile and the digit rows in
-// shared memory into tensor memory, lane i = row i) as soon as the tile has
-// landed, so the pass runs while the warps form the compensator terms; each
-// warp then reads its 32 rows back.  For d = 64 the warps use mma.sync
-// m16n8k32.  Both give the same sums and the same FP32 recombination.
+// per-byte widening is needed.  For d = 128, once the CTAs walk two units or
+// more each, one thread issues them on the fifth-generation tensor cores
+// (tcgen05.mma kind::i8: per 32-column block an M = 128, N = 16, K = 32
+// product from the swizzled tile and the digit rows in shared memory into
+// tensor memory, lane i = row i) as soon as the tile has landed, so the pass
+// runs while the warps form the compensator terms; each warp then reads its
+// 32 rows back.  Otherwise (d = 64, or one unit per CTA, where the tensor
+// memory's allocation and the commit round trip would be pure latency) the
+// warps use mma.sync m16n8k32.  Both give the same sums and the same FP32
+// recombination.
 // Every wait is bounded; an expired wait records LQ_DEVERR_TIMEOUT and all
 // consumer warps leave together at their next barrier.
 #include <cuda.h>
@@ -76,8 +79,10 @@ struct Shape {
     // the INT8 pass on tcgen05 (one thread issues it, the sums land in tensor
     // memory, lane i = row i; d = 128 only), else on warp-level mma.sync
     static constexpr bool TC = TCP && (D == 128);
-    // consumer scratch, in floats: digits (8 x D int8), block scales, vectors,
-    // products, coefficients (two buffers), compensator dots, reductions
+    // consumer scratch, in floats: digits (8 x D int8; with the tensor-core pass
+    // 16 rows of D in its swizzled operand layout, 8 of them zero), block
+    // scales, vectors, products, coefficients (two buffers), compensator dots,
+    // reductions
     static constexpr int RED = 1 + 2 * 8;                          // kq, then (k, q) dots of 8 row comps
     static constexpr int S_B8 = 0, S_EXP = S_B8 + (TC ? 4 * D : 2 * D), S_XQ = S_EXP + 8, S_XK = S_XQ + D, S_QR = S_XK + D,
                          S_KR = S_QR + D, S_A = S_KR + D, S_B = S_A + D, S_CF = S_B + D,
@@ -191,8 +196,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-// Exact int -> float for |x| < 2^22 without the conversion unit: at 1.5 * 2^23
-// the float spacing is 1, so the word 0x4B400000 + x is the number 1.5 * 2^23 + x.
 // tcgen05 pieces of the d = 128 INT8 pass.  Both operands are K-major with
 // 128-byte swizzle: rows of 128 int8 (one row of the state tile, or one digit
 // column), 8-row groups 1024 B apart, 16-byte pieces permuted by the row's
@@ -216,6 +219,8 @@ __device__ __forceinline__ int sw128_off(int row, int kbyte) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// Exact int -> float for |x| < 2^22 without the conversion unit: at 1.5 * 2^23
+// the float spacing is 1, so the word 0x4B400000 + x is the number 1.5 * 2^23 + x.
 __device__ __forceinline__ float i2f_exact(int x) { return __int_as_float(0x4B400000 + x) - 12582912.0f; }
 
 // 2^k as a float, for |k| <= 126.
