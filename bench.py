@@ -380,6 +380,20 @@ def run_e2e(win, wl, dev, L: int, W: int, K: int, args, world: int) -> dict:
                     "pinned host inputs copied in and outputs copied out every token on separate streams"}
 
 
+def bench_config(wl, layers: int, world: int) -> dict:
+    """The `config` of the bench line, the same for both arms."""
+    d, W = wl.d_k, wl.window
+    return {"workload": wl.name, "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
+            "heads": wl.heads, "d_k": d, "d_v": d, "window": W, "n_comp": wl.n_comp_rows + wl.n_comp_cols,
+            "gate": "per-key-channel (KDA)" if wl.per_channel_gate else "scalar (GDN)",
+            "state": "int8 + fp32 buffer",
+            "inputs": "bf16 q/k/v, fp32 g/beta" if wl.dtype == torch.bfloat16 else "fp32",
+            "layers_rotated": layers,
+            "step": f"one window per layer: {W} decode launches + 1 flush, x{layers} layers",
+            "l2": f"not flushed; {layers} layer-states rotated, working set > L2",
+            "parallelism": f"dp{world} (independent sequences per GPU, no collective)"}
+
+
 def run_ours(args, rank, world, local):
     from recurrent_state_quantization_lq_b200 import lq
     dev = torch.device("cuda", local)
@@ -509,14 +523,7 @@ def run_ours(args, rank, world, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": WU,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
-                   "heads": wl.heads, "d_k": d, "d_v": d, "window": W, "n_comp": ncr + ncc,
-                   "gate": "per-key-channel (KDA)" if kda else "scalar (GDN)", "state": "int8 + fp32 buffer",
-                   "inputs": "bf16 q/k/v, fp32 g/beta" if in_b == 2 else "fp32",
-                   "layers_rotated": L,
-                   "step": f"one window per layer: {W} decode launches + 1 flush, x{L} layers",
-                   "l2": f"not flushed; {L} layer-states rotated, working set > L2",
-                   "parallelism": f"dp{world} (independent sequences per GPU, no collective)"},
+        "config": bench_config(wl, L, world),
         "hbm_gbs": achieved,
         "decode_ms_per_step": dec_ms / K, "flush_ms_per_step": fl_ms / K,
         "flush_gbs": fl_bytes / (fl_ms * 1e-3) / 1e9,
@@ -833,8 +840,7 @@ def run_reference(args, rank, world):
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "heads": wl.heads, "d_k": wl.d_k,
-                       "window": wl.window, "n_comp": wl.n_comp_rows + wl.n_comp_cols},
+            "config": bench_config(wl, args.layers, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
