@@ -57,6 +57,12 @@ MUTATIONS = {
     "smoothing factors not applied when decoding": (
         "S[i * dk + j] = (double)sigma[i] * (double)Q[i * dk + j] * (double)s[j];",
         "S[i * dk + j] = (double)sigma[i] * (double)Q[i * dk + j];"),
+    "smoothing multiplied in where it should divide": (
+        "for (int j = 0; j < dk; ++j) rs[j] = 1.0f / s[j];",
+        "for (int j = 0; j < dk; ++j) rs[j] = s[j];"),
+    "row scale applied as a division by 127/M": (
+        "code = rintf((R[i * dk + j] * rs[j]) * rho);",
+        "code = rintf((R[i * dk + j] * rs[j]) / rho);"),
     "smoothing in the naive mode": (
         "const int sm = naive ? 0 : p->smooth;",
         "const int sm = p->smooth;"),

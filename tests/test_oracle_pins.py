@@ -243,6 +243,62 @@ def test_codec_power_of_two_scale_invariance():
     np.testing.assert_array_equal(2 * e1.sigma, e4.sigma)
 
 
+def _definition_quantizer(S, comp_rows, comp_cols, smooth):
+    """The codec's quantizer written as its definition, in FP64, from the FP32
+    residual R (the state with the compensator rows and columns zeroed):
+    s_j = sqrt(max_i |R_ij|) (1 for an empty column, or without smoothing),
+    R' = R / s, sigma_i = max_j |R'_ij| / 127, Q = clamp(rint(R' / sigma), +-127)
+    with Q_i = 0 where sigma_i = 0.  Nothing here calls the oracle."""
+    R = S.astype(np.float32).astype(np.float64)
+    R[list(comp_rows), :] = 0.0
+    R[:, list(comp_cols)] = 0.0
+    m = np.abs(R).max(axis=0)
+    s = np.where((m > 0) & bool(smooth), np.sqrt(m), 1.0)
+    Rp = R / s[None, :]
+    sigma = np.abs(Rp).max(axis=1) / 127.0
+    with np.errstate(divide="ignore", invalid="ignore"):
+        Q = np.where(sigma[:, None] > 0, np.rint(Rp / sigma[:, None]), 0.0)
+    return np.clip(Q, -127, 127).astype(np.int32), sigma, s
+
+
+@pytest.mark.parametrize("smooth", [0, 1])
+@pytest.mark.parametrize("kind", ["normal", "scaled", "planted"])
+def test_quantizer_reading_within_the_definition_bar(kind, smooth):
+    """The oracle applies 1/s_j and 127/M_i as FP32 reciprocal products; the
+    definition divides.  Both must give the same codes within the parity bar of
+    the method (>= 99.9 % equal, never more than 1 LSB apart) and the same
+    scales to FP32 rounding, on normal states, rows spanning six decades
+    (with an empty column) and planted outliers."""
+    from recurrent_state_quantization_lq_b200 import inputs
+    rng = np.random.default_rng(21 + smooth)
+    d = 128
+    cases = []
+    for n in range(6):
+        if kind == "normal":
+            S = rng.standard_normal((d, d))
+        elif kind == "scaled":
+            S = rng.standard_normal((d, d)) * np.logspace(-3, 3, d)[rng.permutation(d)][:, None]
+            S[:, 3] = 0.0
+        else:
+            S = inputs.planted_state(40 + n, 1, 1, d, d)[0][0, 0].double().numpy()
+        cases.append(S)
+    equal, total, worst = 0, 0, 0
+    for S in cases:
+        for nr, nc in ((2, 2), (0, 0), (4, 4)):
+            p = Params(d_k=d, d_v=d, n_comp_rows=nr, n_comp_cols=nc, smooth=smooth)
+            e = oracle.encode(p, S)
+            Qd, sig_d, s_d = _definition_quantizer(S, e.comp_rows, e.comp_cols, smooth)
+            diff = np.abs(e.Q.astype(np.int32) - Qd)
+            equal += int((diff == 0).sum())
+            total += diff.size
+            worst = max(worst, int(diff.max()))
+            # s_j is a correctly rounded square root of an FP32 value: exact
+            np.testing.assert_array_equal(e.s, s_d.astype(np.float32))
+            np.testing.assert_allclose(e.sigma, sig_d, rtol=1e-6, atol=0)
+    assert worst <= 1, worst
+    assert equal / total >= 0.999, equal / total
+
+
 def test_planted_outliers_selected():
     """N(0,1) state with 2 rows and 2 columns x50: L2 ranking finds all four."""
     from recurrent_state_quantization_lq_b200 import inputs
