@@ -282,7 +282,7 @@ def fp32_prefill(wl, n_layers, device, seed):
         tb = inputs.tokens_on_device(seed * 100 + 50 + l, wl.prefill_tokens, wl.batch, wl.heads, wl.d_k, wl.d_v,
                                      wl.per_channel_gate, wl.dtype, device)
         st.prefill_tokens(tb.q, tb.k, tb.v, tb.g, tb.beta)
-        S.append(st.view("state_f32").clone())
+        S.append(st.read("state_f32", device=st.device))
         del st, tb
     torch.cuda.synchronize()
     return S
@@ -765,7 +765,7 @@ def prefill_timing(dev, wl, T: int | None = None, reps: int = 5) -> list[dict]:
         f32.prefill(None)
         for t in range(T):
             f32.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=out[t])
-        win.prefill(f32.view("state_f32"))
+        win.prefill(f32.read("state_f32", device=f32.device))
 
     rows = []
     flop = (6 + (1 if wl.per_channel_gate else 0)) * d * d          # per token and head

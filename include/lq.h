@@ -2,10 +2,22 @@
  * liblq: windowed INT8 recurrent-state decode for gated delta-rule linear
  * attention on NVIDIA B200 (sm_100a).  C ABI.
  *
- * The method (LeapQuant, arXiv 2609.38166; "LeapQuant: Efficient Linear
- * Attention with Accurate Recurrent State Quantization", section "Abstract
- * (arXiv)"): each (sequence, head) pair of a Gated DeltaNet (GDN) or Kimi
- * Delta Attention (KDA) layer keeps a d_v x d_k recurrent state S.  The state
+ * Sources.  Each declaration below names the passage that defines what it
+ * computes:
+ *   [abs]  the paper page "LeapQuant: Efficient Linear Attention with
+ *          Accurate Recurrent State Quantization" (mlsanity.com), section
+ *          "Abstract (arXiv)";
+ *   [news] the bedrocknews.com article on arXiv 2609.38166v1, its paragraph
+ *          on the mechanism (FP32 inference as the baseline, naive per-token
+ *          quantization as the failing alternative, outlier rows and columns
+ *          kept in FP16/FP32).
+ * The pages define no programming interface.  Calls that only manage memory,
+ * handles, errors or checkpoints say "Source: none" and have no counterpart
+ * in the pages.
+ *
+ * The method (LeapQuant, arXiv 2609.38166, [abs]): each (sequence, head)
+ * pair of a Gated DeltaNet (GDN) or Kimi Delta Attention (KDA) layer keeps a
+ * d_v x d_k recurrent state S.  The state
  * is stored as 8-bit codes and is quantized only once per window of W tokens;
  * within a window, outputs come from the fixed low-bit state together with
  * high-precision buffered updates.  The largest outlier rows and columns of
@@ -34,7 +46,7 @@
  *    metadata.  Inputs are read during the call's kernels and not retained.
  *  - Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  All
  *    device work is enqueued on it, asynchronously; no call synchronizes except
- *    lq_device_status().
+ *    lq_device_status() and lq_state_export().
  *  - Errors.  Every call returns an lq_status.  Errors found on the host are
  *    returned at once and leave the state untouched; the text of the last one
  *    on the calling thread is lq_last_error_string().  Errors found on the
@@ -50,7 +62,8 @@
  *    steps, join and leave independently (continuous batching); see
  *    lq_decode_step_active(), lq_window_flush(), lq_window_flush_pending()
  *    and lq_prefill_sequences().
- *  - Threads.  A handle must not be used by two threads at once.
+ *  - Threads.  A handle must not be used by two threads at once; different
+ *    handles may be used from different host threads concurrently.
  */
 #ifndef LQ_H
 #define LQ_H
@@ -137,16 +150,22 @@ typedef struct lq_layout {
 
 typedef struct lq_state_s *lq_handle;
 
-/* Bytes of device workspace a config needs; 0 if the config is invalid. */
+/* Bytes of device workspace a config needs; 0 if the config is invalid.
+ * Source: none (memory sizing). */
 LQ_API size_t lq_workspace_bytes(const lq_config *cfg);
 
-/* Fill *out with the workspace layout of a valid config. */
+/* Fill *out with the workspace layout of a valid config.  The layout is
+ * internal and may change between versions: read the state through
+ * lq_state_export(); use the layout only to checkpoint whole workspaces.
+ * Source: none (memory layout). */
 LQ_API lq_status lq_workspace_layout(const lq_config *cfg, lq_layout *out);
 
 /*
  * Create a handle over a caller-owned workspace (d_workspace: device pointer,
  * 256-byte aligned, `bytes` >= lq_workspace_bytes(cfg)).  Host-only: touches
  * no device memory.  The state is undefined until lq_prefill_state().
+ * Source: [abs] (one recurrent state per (sequence, head) of a GDN or KDA
+ * layer, held in 8 bits); the handle itself has no counterpart.
  */
 LQ_API lq_status lq_state_create(const lq_config *cfg, void *d_workspace, size_t bytes, lq_handle *out);
 
@@ -159,6 +178,9 @@ LQ_API lq_status lq_state_create(const lq_config *cfg, void *d_workspace, size_t
  *   naive:    per-row INT8 without compensators or smoothing;
  *   FP32:     a copy.
  * Clears the error word, the gate sums and the window buffer.
+ * Source: [abs] (the state is quantized once per window, at its end, with
+ * the largest outliers kept as Compensator Tokens and the residual smoothed
+ * before quantization); [news] for the naive and FP32 comparators.
  */
 LQ_API lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream);
 
@@ -174,6 +196,9 @@ LQ_API lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream);
  * state; it returns LQ_ERR_WINDOW_FULL when W tokens are already buffered.
  * Naive mode updates and requantizes the INT8 state; FP32 mode updates it.
  * On a ragged handle this is lq_decode_step_active() with every sequence active.
+ * Source: [abs] (outputs from the fixed low-bit state plus high-precision
+ * buffered updates; Compensator Tokens on the update path of real tokens);
+ * [news] (the FP32-state baseline and naive per-token quantization).
  */
 LQ_API lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, const void *d_v,
                          const float *d_g, const float *d_beta, float *d_o, void *stream);
@@ -186,6 +211,10 @@ LQ_API lq_status lq_decode_step(lq_handle h, const void *d_q, const void *d_k, c
  * unit whose window already holds W tokens is skipped and LQ_DEVERR_WINDOW_FULL
  * recorded (lq_device_status() returns LQ_ERR_WINDOW_FULL): call
  * lq_window_flush() after every step.  LQ_ERR_STATE on a shared-phase handle.
+ * The beta and g entries of inactive sequences may be read (a prefetch) but
+ * never affect any result; their q, k, v rows are not read.
+ * Source: [abs] (the windowed scheme, applied to each sequence over its own
+ * tokens; the pages do not discuss sequences that join or skip steps).
  */
 LQ_API lq_status lq_decode_step_active(lq_handle h, const void *d_q, const void *d_k, const void *d_v,
                                        const float *d_g, const float *d_beta, const uint8_t *d_active,
@@ -204,12 +233,16 @@ LQ_API lq_status lq_decode_step_active(lq_handle h, const void *d_q, const void 
  * launches nothing when no window is full and otherwise flushes like a
  * shared-phase handle.  Once phases differ, a launch reads every unit's count
  * and re-encodes only the due units.
+ * Source: [abs] (quantized a single time, at the end of the window; largest
+ * outliers kept as high-precision Compensator Tokens; residual smoothed
+ * before quantization); [news] (the outliers are whole rows and columns).
  */
 LQ_API lq_status lq_window_flush(lq_handle h, void *stream);
 
 /*
  * Ragged handles: flush every unit holding at least one buffered token (for
  * example before a sequence leaves).  Shared-phase handles: lq_window_flush().
+ * Source: [abs], as lq_window_flush() (a window that ends early).
  */
 LQ_API lq_status lq_window_flush_pending(lq_handle h, void *stream);
 
@@ -219,6 +252,7 @@ LQ_API lq_status lq_window_flush_pending(lq_handle h, void *stream);
  * [batch][heads][d_v][d_k], only their rows read; NULL = all-zero state) and
  * their windows emptied; the other sequences are untouched.  Requires a prior
  * lq_prefill_state(); LQ_ERR_STATE on a shared-phase handle.
+ * Source: [abs], as lq_prefill_state().
  */
 LQ_API lq_status lq_prefill_sequences(lq_handle h, const float *d_S0, const uint8_t *d_mask, void *stream);
 
@@ -241,6 +275,8 @@ LQ_API lq_status lq_prefill_sequences(lq_handle h, const float *d_S0, const uint
  * phases are aligned).  The caller keeps ownership of every buffer; nothing is
  * retained after the call.  Errors: LQ_ERR_INVALID_ARG for a NULL input with
  * n_tokens > 0, a negative n_tokens or a misaligned pointer.
+ * Source: [abs] (the codec once, at the end of the prompt; the pages do not
+ * say how a prompt is ingested, so the prompt itself runs in FP32).
  */
 LQ_API lq_status lq_prefill_tokens(lq_handle h, const float *d_S0, const void *d_q, const void *d_k,
                                    const void *d_v, const float *d_g, const float *d_beta, int32_t n_tokens,
@@ -260,6 +296,7 @@ LQ_API lq_status lq_prefill_tokens(lq_handle h, const float *d_S0, const void *d
  * lq_prefill_state(); LQ_ERR_STATE on a shared-phase handle; LQ_ERR_INVALID_ARG
  * for a NULL mask, a negative max_tokens, a NULL input with max_tokens > 0 or a
  * misaligned pointer.
+ * Source: [abs], as lq_prefill_tokens().
  */
 LQ_API lq_status lq_prefill_sequences_tokens(lq_handle h, const float *d_S0, const void *d_q, const void *d_k,
                                              const void *d_v, const float *d_g, const float *d_beta,
@@ -278,23 +315,68 @@ LQ_API lq_status lq_prefill_sequences_tokens(lq_handle h, const float *d_S0, con
  * from the workspace and ignores n_buf (pass 0).  No device work; the next
  * decode, flush or prefill continues exactly where the checkpoint stood.
  * Errors: LQ_ERR_INVALID_ARG for a bad handle or an n_buf out of range.
+ * Source: none (checkpointing).
  */
 LQ_API lq_status lq_state_resume(lq_handle h, int32_t n_buf);
 
+/*
+ * Destination buffers of lq_state_export(), N = batch * heads units in
+ * (sequence, head) order, each region packed with no padding.  Every pointer
+ * may be NULL (that region is not copied) or point to device memory or to
+ * host memory (pinned or pageable); the caller owns them.  A non-NULL pointer
+ * for a region the handle's mode does not keep is an error.
+ */
+typedef struct lq_export {
+    int8_t *codes;          /* int8  [N][d_v][d_k]   Q             windowed, naive */
+    float *row_scale;       /* f32   [N][d_v]        sigma         windowed, naive */
+    float *col_smooth;      /* f32   [N][d_k]        s             windowed        */
+    int32_t *comp_index;    /* int32 [N][n_comp_rows + n_comp_cols]: rows, columns */
+    float *comp_row_vec;    /* f32   [N][n_comp_rows][d_k]  k of row compensators  */
+    float *comp_col_vec;    /* f32   [N][n_comp_cols][d_v]  v of column comps      */
+    float *buf_delta;       /* f32   [N][window][d_v]  buffered delta_j            */
+    void *buf_key;          /* [N][window][d_k]: GDN in_dtype k_j; KDA f32
+                               k_j * exp(-G_j)                                     */
+    float *buf_gate;        /* f32   [N][window]  exp(-G_j) of entry j (GDN)       */
+    double *gate_sum;       /* f64   [N][1 (GDN) or d_k (KDA)]: G of the window    */
+    int32_t *fill;          /* int32 [N] tokens buffered per unit, 0..W (windowed
+                               mode, shared or ragged phases)                      */
+    float *state_f32;       /* f32   [N][d_v][d_k]                 FP32 mode       */
+} lq_export;
+
+/*
+ * Copy the current state into caller buffers (see lq_export): the stored
+ * window-start state (codes, row scales, smoothing factors, Compensator
+ * Tokens), the window's buffered entries and their count, or the FP32 state.
+ * Buffer entries past a unit's count are copied but hold no meaning.
+ * Enqueues the copies on `stream`, then synchronizes it (like
+ * lq_device_status()) and reads the device error word.  Returns LQ_OK; the
+ * device status (LQ_ERR_RANGE, LQ_ERR_WINDOW_FULL or LQ_ERR_DEVICE, text in
+ * lq_last_error_string()) when the error word is set, in which case the
+ * copied state may be inconsistent; LQ_ERR_INVALID_ARG for a bad handle, a
+ * NULL dst or a pointer for an absent region (nothing is copied);
+ * LQ_ERR_STATE before lq_prefill_state(); LQ_ERR_CUDA when a copy fails.
+ * Source: [abs] (the fixed low-bit state: 8-bit codes plus high-precision
+ * buffered updates and Compensator Tokens); [news] for the FP32 state.
+ */
+LQ_API lq_status lq_state_export(lq_handle h, const lq_export *dst, void *stream);
+
 /* Tokens buffered in the current window (0..W); -1 for a bad or ragged handle
- * (a ragged handle's counts are on the device, at lq_layout.fill). */
+ * (a ragged handle's counts are on the device: lq_state_export() reads them).
+ * Source: [abs] (the window of W tokens). */
 LQ_API int32_t lq_window_fill(lq_handle h);
 
 /*
- * Synchronize `stream` and read the device error word: LQ_OK, LQ_ERR_RANGE or
- * LQ_ERR_DEVICE (detail in lq_last_error_string()).
+ * Synchronize `stream` and read the device error word: LQ_OK, LQ_ERR_RANGE,
+ * LQ_ERR_WINDOW_FULL or LQ_ERR_DEVICE (detail in lq_last_error_string()).
+ * Source: none (error reporting).
  */
 LQ_API lq_status lq_device_status(lq_handle h, void *stream);
 
-/* Release the handle (host metadata only; the workspace stays the caller's). */
+/* Release the handle (host metadata only; the workspace stays the caller's).
+ * Source: none. */
 LQ_API lq_status lq_state_destroy(lq_handle h);
 
-/* Text of the last error on the calling thread ("" if none). */
+/* Text of the last error on the calling thread ("" if none).  Source: none. */
 LQ_API const char *lq_last_error_string(void);
 
 #ifdef __cplusplus

@@ -6,6 +6,7 @@
 #include <cstring>
 #include <new>
 #include <string>
+#include <vector>
 
 #include "lq.h"
 #include <nvtx3/nvToolsExt.h>
@@ -485,6 +486,71 @@ lq_status lq_prefill_sequences(lq_handle h, const float *d_S0, const uint8_t *d_
     if (e != cudaSuccess) return cuda_fail(e, "launching the encode kernel");
     h->aligned = 0;                       // the restarted sequences start a new phase
     return LQ_OK;
+}
+
+lq_status lq_state_export(lq_handle h, const lq_export *dst, void *stream) {
+    Range nvtx_range("lq_state_export");
+    if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    if (dst == nullptr) return fail(LQ_ERR_INVALID_ARG, "export destinations are NULL");
+    const lq_config &c = h->cfg;
+    const lq_layout &L = h->lay;
+    const size_t N = (size_t)c.batch * c.heads, d = (size_t)c.d_k, W = (size_t)c.window;
+    const size_t gd = (c.gate == LQ_GATE_CHANNEL) ? d : 1;
+    const size_t key_b = (c.gate == LQ_GATE_CHANNEL || c.in_dtype == LQ_DTYPE_F32) ? 4 : 2;
+    const size_t ncomp = (size_t)(c.n_comp_rows + c.n_comp_cols);
+    // (destination, workspace offset, rows, packed row bytes, workspace row pitch)
+    struct Region {
+        void *dst;
+        size_t off, rows, row_bytes, pitch;
+        const char *name;
+    };
+    const Region regions[] = {
+        {dst->codes, L.codes, N, d * d, d * d, "codes"},
+        {dst->row_scale, L.row_scale, N, d * 4, d * 4, "row_scale"},
+        {dst->col_smooth, L.col_smooth, N, d * 4, d * 4, "col_smooth"},
+        {dst->comp_index, L.comp_index, N, ncomp * 4, (size_t)L.comp_index_stride * 4, "comp_index"},
+        {dst->comp_row_vec, L.comp_row_vec, N, (size_t)c.n_comp_rows * d * 4, (size_t)c.n_comp_rows * d * 4,
+         "comp_row_vec"},
+        {dst->comp_col_vec, L.comp_col_vec, N, (size_t)c.n_comp_cols * d * 4, (size_t)c.n_comp_cols * d * 4,
+         "comp_col_vec"},
+        {dst->buf_delta, L.buf_delta, N, W * d * 4, W * d * 4, "buf_delta"},
+        {dst->buf_key, L.buf_key, N, W * d * key_b, W * d * key_b, "buf_key"},
+        {dst->buf_gate, L.buf_gate, N, W * 4, (size_t)L.window_pad * 4, "buf_gate"},
+        {dst->gate_sum, L.gate_sum, N, gd * 8, gd * 8, "gate_sum"},
+        {dst->state_f32, L.state_f32, N, d * d * 4, d * d * 4, "state_f32"},
+    };
+    // every requested region must exist before anything is copied
+    for (const Region &r : regions)
+        if (r.dst != nullptr && r.off == LQ_ABSENT)
+            return fail(LQ_ERR_INVALID_ARG, std::string("this handle's mode keeps no ") + r.name);
+    if (dst->fill != nullptr && c.mode != LQ_MODE_WINDOW)
+        return fail(LQ_ERR_INVALID_ARG, "this handle's mode keeps no window counts");
+    if (!h->prefilled) return fail(LQ_ERR_STATE, "export before lq_prefill_state");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    for (const Region &r : regions) {
+        if (r.dst == nullptr || r.row_bytes == 0) continue;
+        if (r.row_bytes == r.pitch)
+            e = cudaMemcpyAsync(r.dst, h->ws + r.off, r.rows * r.row_bytes, cudaMemcpyDefault, s);
+        else
+            e = cudaMemcpy2DAsync(r.dst, r.row_bytes, h->ws + r.off, r.pitch, r.row_bytes, r.rows, cudaMemcpyDefault,
+                                  s);
+        if (e != cudaSuccess) return cuda_fail(e, (std::string("exporting ") + r.name).c_str());
+    }
+    // window counts: on the device for ragged handles, else the handle's shared count
+    std::vector<int32_t> shared_fill;
+    if (dst->fill != nullptr) {
+        if (c.ragged) {
+            e = cudaMemcpyAsync(dst->fill, h->ws + L.fill, N * 4, cudaMemcpyDefault, s);
+        } else {
+            shared_fill.assign(N, h->n_buf);
+            e = cudaMemcpyAsync(dst->fill, shared_fill.data(), N * 4, cudaMemcpyDefault, s);
+        }
+        if (e != cudaSuccess) return cuda_fail(e, "exporting the window counts");
+    }
+    // drains the stream (the host count buffer stays alive until then) and
+    // reports the error word
+    return lq_device_status(h, stream);
 }
 
 lq_status lq_device_status(lq_handle h, void *stream) {

@@ -49,6 +49,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "lq_decode_parts.cuh"
 #include "lq_kernels.h"
 
 namespace lq {
@@ -62,9 +63,9 @@ constexpr int kSlots = 3;
 constexpr int kCtasPerSm = 4;
 constexpr int kConsumerBarrier = 1;           // named barrier of the consumer warps
 constexpr int kPer = 4;                       // buffered entries per warp per chunk
-constexpr double kMaxAbsGateSum = 80.0;
+using namespace dec;
 
-__host__ __device__ constexpr int align_up(int x, int a) { return (x + a - 1) / a * a; }
+__device__ __forceinline__ bool consumer_sync_or(bool pred) { return named_sync_or(kConsumerBarrier, kConsumers, pred); }
 
 template <int D, bool KDA, typename InT, typename KeyT, bool TCP>
 struct Shape {
@@ -94,164 +95,6 @@ struct Shape {
     static_assert(MT >= 1, "m-tiles");
 };
 
-// Offsets inside a meta segment.
-struct Meta {
-    int sig, s, qin, kin, vin, gin, gsum, cidx, crow, ccol, bytes;
-};
-
-template <int D, bool KDA, typename InT>
-__host__ __device__ Meta meta_layout(int ncr, int ncc, int cis) {
-    Meta m{};
-    int o = 0;
-    m.sig = o;  o += 4 * D;
-    m.s = o;    o += 4 * D;
-    m.qin = o;  o += (int)sizeof(InT) * D;
-    m.kin = o;  o += (int)sizeof(InT) * D;
-    m.vin = o;  o += (int)sizeof(InT) * D;
-    m.gin = o;  o += KDA ? 4 * D : 0;
-    m.gsum = o; o += KDA ? 8 * D : 0;
-    m.cidx = o; o += (ncr + ncc) > 0 ? 4 * cis : 0;
-    m.crow = o; o += 4 * D * ncr;
-    m.ccol = o; o += 4 * D * ncc;
-    m.bytes = o;
-    return m;
-}
-
-template <typename T>
-__device__ __forceinline__ float to_f32(T x) { return static_cast<float>(x); }
-template <>
-__device__ __forceinline__ float to_f32<float>(float x) { return x; }
-
-template <typename KeyT, int VPL>
-__device__ __forceinline__ void load_key(const KeyT *p, float (&out)[VPL]) {
-    if constexpr (sizeof(KeyT) == 2) {
-        if constexpr (VPL == 4) {
-            uint2 w = *reinterpret_cast<const uint2 *>(p);
-            out[0] = bf16_bits_to_f32(w.x & 0xffffu); out[1] = bf16_bits_to_f32(w.x >> 16);
-            out[2] = bf16_bits_to_f32(w.y & 0xffffu); out[3] = bf16_bits_to_f32(w.y >> 16);
-        } else {
-            uint32_t w = *reinterpret_cast<const uint32_t *>(p);
-            out[0] = bf16_bits_to_f32(w & 0xffffu); out[1] = bf16_bits_to_f32(w >> 16);
-        }
-    } else {
-        if constexpr (VPL == 4) {
-            float4 w = *reinterpret_cast<const float4 *>(p);
-            out[0] = w.x; out[1] = w.y; out[2] = w.z; out[3] = w.w;
-        } else {
-            float2 w = *reinterpret_cast<const float2 *>(p);
-            out[0] = w.x; out[1] = w.y;
-        }
-    }
-}
-
-// Consumer barrier that also ORs a predicate over the consumer threads.
-__device__ __forceinline__ bool consumer_sync_or(bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(kConsumerBarrier), "r"(kConsumers)
-        : "memory");
-    return r != 0;
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Byte offset of the 16-byte chunk `chunk` of row `row` in a D x D int8 tile
-// written by the tensor copy with the 128-byte (D = 128) or 64-byte (D = 64)
-// swizzle: the chunk index is XORed with address bits 7-9 (resp. 7-8).
-template <int D>
-__device__ __forceinline__ int swz(int row, int chunk) {
-    if constexpr (D == 128) return row * 128 + ((chunk ^ (row & 7)) << 4);
-    else return row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4);
-}
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-
-// D (16x8 s32) += A (16x32 s8, row) * B (32x8 s8, col)
-__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                       uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// 2-D tensor copy of the (x, y) box of `map` into shared memory.
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// tcgen05 pieces of the d = 128 INT8 pass.  Both operands are K-major with
-// 128-byte swizzle: rows of 128 int8 (one row of the state tile, or one digit
-// column), 8-row groups 1024 B apart, 16-byte pieces permuted by the row's
-// index mod 8 -- the layout the tile's 2-D tensor copy writes.
-constexpr int kTmemCols = 64;                 // 4 blocks x 16 accumulator columns
-// s32 accumulator, s8 A and B, both K-major, N = 16, M = 128
-constexpr uint32_t kI8Idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
-
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr >> 4) & 0x3fff);   // start address
-    d |= (uint64_t)(16 >> 4) << 16;           // leading byte offset (unused with this swizzle)
-    d |= (uint64_t)(1024 >> 4) << 32;         // stride byte offset: 8-row groups
-    d |= (uint64_t)1 << 46;                   // descriptor version
-    d |= (uint64_t)2 << 61;                   // 128-byte swizzle
-    return d;
-}
-__device__ __forceinline__ int sw128_off(int row, int kbyte) {
-    return (row >> 3) * 1024 + (row & 7) * 128 + ((((kbyte >> 4) ^ (row & 7))) << 4) + (kbyte & 15);
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Exact int -> float for |x| < 2^22 without the conversion unit: at 1.5 * 2^23
-// the float spacing is 1, so the word 0x4B400000 + x is the number 1.5 * 2^23 + x.
-__device__ __forceinline__ float i2f_exact(int x) { return __int_as_float(0x4B400000 + x) - 12582912.0f; }
-
-// 2^k as a float, for |k| <= 126.
-__device__ __forceinline__ float pow2i(int k) { return __int_as_float((127 + k) << 23); }
-
-// Block exponent of a block with maximum |y| = m: 2^E with m 2^-E in [32, 64),
-// returned as (2^-E, 2^E); (0, 0) for a block too small to matter.
-__device__ __forceinline__ float2 block_scale(float m) {
-    const int biased = (__float_as_int(m) >> 23) & 0xff;     // m = 1.f x 2^(biased - 127)
-    if (biased < 20) return make_float2(0.0f, 0.0f);          // |y| < 2^-107 (or zero)
-    const int E = biased - 127 + 1 - 6;
-    return make_float2(pow2i(-E), pow2i(E));
-}
-
-// The four base-2^7 int8 digits of y * 2^-E (|y 2^-E| < 64), packed low to high.
-// Every |r| here is at most 64, so adding 1.5 * 2^23 rounds r to an integer
-// (to nearest, ties to even, as rintf) with no conversion instruction: the
-// sum minus 1.5 * 2^23 is the digit as a float, and the sum's low byte is its
-// two's-complement byte.
-__device__ __forceinline__ uint32_t digits4(float y, float down) {
-    float r = y * down;
-    uint32_t out = 0;
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const float t = __fadd_rn(r, 12582912.0f);
-        const float d = __fsub_rn(t, 12582912.0f);
-        out |= (__float_as_uint(t) & 0xffu) << (8 * p);
-        r = (r - d) * 128.0f;
-    }
-    return out;
-}
 template <int D, bool KDA, typename InT, typename KeyT, bool RAGGED, bool TCP>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_window_kernel(DecodeArgs a, const __grid_constant__ CUtensorMap codes_map) {
@@ -306,15 +149,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const uint32_t in_b = (uint32_t)sizeof(InT) * D;
         int slot = 0;
         uint32_t ph = 0;
+        uint32_t armed = 0;                        // slots filled at least once
         auto acquire = [&](int u, int detail) -> unsigned char * {
             if (!mbar_wait(&empty[slot], ph ^ 1u, kWaitBudgetCycles)) {
                 report_error(w.err, LQ_DEVERR_TIMEOUT, u, detail);
                 return nullptr;
             }
+            armed |= 1u << slot;
             return ring + slot * kSlotBytes;
         };
         auto advance = [&]() {
             if (++slot == kSlots) { slot = 0; ph ^= 1u; }
+        };
+        // After a timed-out acquire the consumers have stopped: wait (bounded)
+        // until every copy this thread started has landed, so that no copy
+        // still writes into the shared memory of a CTA that has exited.  Slot
+        // i was last filled in the round whose parity is ph for i < slot and
+        // ph ^ 1 for i >= slot.
+        auto drain = [&]() {
+            for (int i = 0; i < kSlots; ++i)
+                if (armed & (1u << i)) mbar_wait(&full[i], i < slot ? ph : (ph ^ 1u), kWaitBudgetCycles);
         };
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
             const int n_buf = unit_fill(u);
@@ -325,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
             const int nchunks = (n_buf + E - 1) / E;
             unsigned char *dst = acquire(u, -1);
-            if (dst == nullptr) return;
+            if (dst == nullptr) { drain(); return; }
             uint64_t *bar = &full[slot];
             mbar_arrive_expect_tx(bar, (uint32_t)M.bytes);
             bulk_g2s(dst + M.sig, w.row_scale + (size_t)u * D, 4 * D, bar);
@@ -344,14 +198,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
             advance();
             dst = acquire(u, -2);
-            if (dst == nullptr) return;
+            if (dst == nullptr) { drain(); return; }
             bar = &full[slot];
             mbar_arrive_expect_tx(bar, D * D);
             tma_load_2d(dst, &codes_map, 0, u * D, bar);
             advance();
             for (int c = 0; c < nchunks; ++c) {
                 dst = acquire(u, -3 - c);
-                if (dst == nullptr) return;
+                if (dst == nullptr) { drain(); return; }
                 const int e0 = c * E, ne = min(E, n_buf - e0);
                 const size_t first = (size_t)u * w.window + e0;
                 const uint32_t bd = 4u * ne * D, bk = (uint32_t)sizeof(KeyT) * ne * D;
@@ -385,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     };
     const uint32_t tmem = Sh::TC ? *tmem_slot : 0u;   // lane i = state row i
     uint32_t mph = 0;                                 // phase of the tcgen05 pass barrier
+    bool tc_inflight = false;                         // a pass was issued and not yet seen complete
     int u = blockIdx.x;
     float beta_n = 0.0f, g_n = 0.0f, gam_n = 0.0f;
     double G_n = 0.0;
@@ -532,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
 
         if constexpr (Sh::TC) {
+            tc_inflight = true;
             // One thread starts the INT8 pass as soon as the tile is in: per
             // 32-column block kb an M = 128, N = 16, K = 32 s8 product into
             // tensor-memory columns 16 kb ..  It runs under the compensator terms.
@@ -591,7 +447,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if constexpr (!Sh::TC) bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
         float p8q = 0.0f, p8k = 0.0f;              // TC: this thread's row of the two products
         if constexpr (Sh::TC) {
-            bad |= !mbar_wait(mma_bar, mph, kWaitBudgetCycles);
+            if (mbar_wait(mma_bar, mph, kWaitBudgetCycles)) tc_inflight = false;
+            else bad = true;
             mph ^= 1u;
             tc_fence_after();
             __syncwarp();
@@ -753,28 +610,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
 consumers_done:
     // every consumer warp gets here (normal end, or a timeout all of them saw at
-    // the same barrier); no tensor-core pass is in flight, so the tensor memory
-    // goes back once all warps' loads are done
+    // the same barrier).  After a timeout a tensor-core pass may still be in
+    // flight: wait for it (bounded) before the tensor memory goes back, once
+    // all warps' loads are done.
     if constexpr (Sh::TC) {
+        if (tc_inflight) mbar_wait(mma_bar, mph ^ 1u, kWaitBudgetCycles);
         tc_fence_before();
         asm volatile("bar.sync %0, %1;" ::"r"(kConsumerBarrier), "r"(kConsumers) : "memory");
         tc_fence_after();
         if (warp == 0)
             asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
-}
-
-int sm_count() {
-    static int cached[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (dev < 0 || dev >= 64) return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
-    }
-    return cached[dev];
 }
 
 template <int D, bool KDA, typename InT, typename KeyT, bool RAGGED, bool TCP>
@@ -785,15 +631,8 @@ cudaError_t launch_r(const DecodeArgs &a, cudaStream_t s) {
     auto kern = decode_window_kernel<D, KDA, InT, KeyT, RAGGED, TCP>;
     // The opt-in shared-memory size is set once per device, so that launches
     // inside a stream capture make no attribute calls.
-    static bool opted_in[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    const cudaError_t e = opt_in_smem<decode_window_kernel<D, KDA, InT, KeyT, RAGGED, TCP>>(Sh::SMEM);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !opted_in[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::SMEM);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) opted_in[dev] = true;
-    }
     const int grid = min(a.w.units, kCtasPerSm * sm_count());
     kern<<<grid, kThreads, Sh::SMEM, s>>>(a, *reinterpret_cast<const CUtensorMap *>(a.codes_map));
     return cudaGetLastError();
@@ -820,14 +659,22 @@ cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t make_codes_map(void *map_out, const int8_t *codes, int d, int units) {
-    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    // the driver's entry point, looked up once (first callers serialized)
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> entry{nullptr};
+    static std::mutex lookup;
+    PFN_cuTensorMapEncodeTiled_v12000 encode = entry.load(std::memory_order_acquire);
     if (encode == nullptr) {
-        void *fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-        if (e != cudaSuccess) return e;
-        if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorNotSupported;
-        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        std::lock_guard<std::mutex> lock(lookup);
+        encode = entry.load(std::memory_order_relaxed);
+        if (encode == nullptr) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+            if (e != cudaSuccess) return e;
+            if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorNotSupported;
+            encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            entry.store(encode, std::memory_order_release);
+        }
     }
     const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)units * (cuuint64_t)d};
     const cuuint64_t strides[1] = {(cuuint64_t)d};

@@ -356,34 +356,14 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
     }
 }
 
-int sm_count() {
-    static int cached[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (dev < 0 || dev >= 64) return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
-    }
-    return cached[dev];
-}
-
 template <int D, bool KDA, typename KeyT>
 cudaError_t launch_flush_t(const EncodeArgs &a, cudaStream_t s) {
     using Sh = FlushShape<D, KDA, KeyT>;
     const FlushMeta M = flush_meta_layout<D, KDA>(a.w.n_comp_rows, a.w.n_comp_cols, a.w.comp_index_stride);
     if (M.bytes > kSlotBytes || D * D > kSlotBytes) return cudaErrorInvalidValue;
     auto kern = flush_kernel<D, KDA, KeyT>;
-    static bool opted_in[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    const cudaError_t e = opt_in_smem<flush_kernel<D, KDA, KeyT>>(Sh::SMEM);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !opted_in[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::SMEM);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) opted_in[dev] = true;
-    }
     const int grid = min(a.w.units, 2 * sm_count());
     kern<<<grid, kFlushThreads, Sh::SMEM, s>>>(a);
     return cudaGetLastError();

@@ -493,22 +493,19 @@ cudaError_t launch_t(const EncodeArgs &a, cudaStream_t s) {
     cfg.numAttrs = 1;
     // Clusters that fit on the GPU at once, found once per device (outside any
     // stream capture: the first flush of a handle runs before graphs are made).
-    static int clusters[64] = {0};
-    int dev = 0;
+    static DeviceCache clusters;
+    int dev = 0, n_clusters = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (clusters[dev] == 0) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        cfg.gridDim = dim3(Sh::C, 1, 1);
-        int n = 0;
-        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
-        if (e != cudaSuccess) return e;
-        if (n <= 0) return cudaErrorInvalidConfiguration;
-        clusters[dev] = n;
-    }
-    const int ncl = min(clusters[dev], a.w.units);
+    e = clusters.get(dev, &n_clusters, [&](int *v) {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (r != cudaSuccess) return r;
+        cudaLaunchConfig_t probe = cfg;
+        probe.gridDim = dim3(Sh::C, 1, 1);
+        return cudaOccupancyMaxActiveClusters(v, kern, &probe);
+    });
+    if (e != cudaSuccess) return e;
+    const int ncl = min(n_clusters, a.w.units);
     cfg.gridDim = dim3((unsigned)(ncl * Sh::C), 1, 1);
     return cudaLaunchKernelEx(&cfg, kern, a);
 }

@@ -4,9 +4,73 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "lq_common.cuh"
 
 namespace lq {
+
+constexpr int kMaxDevices = 64;
+
+// A positive per-device value that a launcher computes on its first call on a
+// device (an occupancy figure, or 1 once a function attribute is set) and then
+// reuses, so that launches inside a stream capture make no runtime queries.
+// Different handles may be driven from different host threads: the first
+// calls on a device are serialized and `make` runs once per device until it
+// succeeds; later calls read the value without taking the lock.
+class DeviceCache {
+  public:
+    template <typename F>
+    cudaError_t get(int dev, int *out, F &&make) {
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        int v = value_[dev].load(std::memory_order_acquire);
+        if (v <= 0) {
+            std::lock_guard<std::mutex> lock(mutex_);
+            v = value_[dev].load(std::memory_order_relaxed);
+            if (v <= 0) {
+                const cudaError_t e = make(&v);
+                if (e != cudaSuccess) return e;
+                if (v <= 0) return cudaErrorInvalidConfiguration;
+                value_[dev].store(v, std::memory_order_release);
+            }
+        }
+        *out = v;
+        return cudaSuccess;
+    }
+
+  private:
+    std::atomic<int> value_[kMaxDevices] = {};
+    std::mutex mutex_;
+};
+
+// Streaming multiprocessors of the current device (148 on a B200 if the query
+// fails).
+inline int sm_count() {
+    static DeviceCache cache;
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    const cudaError_t e = cache.get(dev, &n, [dev](int *v) {
+        if (cudaDeviceGetAttribute(v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || *v <= 0) *v = 148;
+        return cudaSuccess;
+    });
+    return e == cudaSuccess ? n : 148;
+}
+
+// Set a kernel's dynamic shared-memory limit once per device (one cache per
+// kernel: the template is keyed on the kernel's address, not on its type).
+template <auto kern>
+cudaError_t opt_in_smem(int bytes) {
+    static DeviceCache cache;
+    int dev = 0, done = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    return cache.get(dev, &done, [&](int *v) {
+        const cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        *v = 1;
+        return r;
+    });
+}
 
 struct EncodeArgs {
     Views w;

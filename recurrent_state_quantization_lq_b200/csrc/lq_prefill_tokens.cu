@@ -349,15 +349,8 @@ cudaError_t launch_t(const TokenPrefillArgs &a, cudaStream_t s) {
     using Sh = TokShape<D, KDA, (int)sizeof(InT)>;
     auto kern = prefill_tokens_kernel<D, KDA, InT>;
     const int smem = 4 * Sh::WORDS;
-    static bool opted_in[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    const cudaError_t e = opt_in_smem<prefill_tokens_kernel<D, KDA, InT>>(smem);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !opted_in[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) opted_in[dev] = true;
-    }
     kern<<<a.w.units, Sh::NT, smem, s>>>(a);
     return cudaGetLastError();
 }

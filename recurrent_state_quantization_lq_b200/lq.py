@@ -44,6 +44,15 @@ class Layout(ctypes.Structure):
         [("comp_index_stride", ctypes.c_int32), ("window_pad", ctypes.c_int32), ("fill", ctypes.c_size_t)]
 
 
+EXPORT_REGIONS = ("codes", "row_scale", "col_smooth", "comp_index", "comp_row_vec", "comp_col_vec", "buf_delta",
+                  "buf_key", "buf_gate", "gate_sum", "fill", "state_f32")
+
+
+class Export(ctypes.Structure):
+    """lq_export: destination pointers of lq_state_export (NULL = not copied)."""
+    _fields_ = [(n, ctypes.c_void_p) for n in EXPORT_REGIONS]
+
+
 class LQError(RuntimeError):
     def __init__(self, status: int, what: str):
         super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}: {last_error()}")
@@ -88,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.lq_state_resume.restype = i32
         L.lq_window_fill.argtypes = [vp]
         L.lq_window_fill.restype = i32
+        L.lq_state_export.argtypes = [vp, ctypes.POINTER(Export), vp]
+        L.lq_state_export.restype = i32
         L.lq_device_status.argtypes = [vp, vp]
         L.lq_device_status.restype = i32
         L.lq_state_destroy.argtypes = [vp]
@@ -286,8 +297,61 @@ class DecodeState:
         return lib().lq_window_fill(self._h)
 
     def fills(self) -> torch.Tensor:
-        """Ragged: tokens buffered per (sequence, head), read from the device."""
-        return self.view("fill").clone()
+        """Tokens buffered per (sequence, head) (read through lq_state_export,
+        whatever the device error word holds)."""
+        return self.export(["fill"], check=False)["fill"]
+
+    def export_shapes(self) -> dict:
+        """Dtype and packed shape of every region lq_state_export can copy for
+        this state (regions the mode does not keep are absent)."""
+        L, c = self.layout, self.cfg
+        B, H, d, W = c.batch, c.heads, c.d_k, c.window
+        key_dt = torch.float32 if (c.gate == 1 or c.in_dtype == 0) else torch.bfloat16
+        spec = {
+            "codes": (torch.int8, (B, H, d, d)),
+            "row_scale": (torch.float32, (B, H, d)),
+            "col_smooth": (torch.float32, (B, H, d)),
+            "comp_index": (torch.int32, (B, H, c.n_comp_rows + c.n_comp_cols)),
+            "comp_row_vec": (torch.float32, (B, H, c.n_comp_rows, d)),
+            "comp_col_vec": (torch.float32, (B, H, c.n_comp_cols, d)),
+            "buf_delta": (torch.float32, (B, H, W, d)),
+            "buf_key": (key_dt, (B, H, W, d)),
+            "buf_gate": (torch.float32, (B, H, W)),
+            "gate_sum": (torch.float64, (B, H, d if c.gate == 1 else 1)),
+            "fill": (torch.int32, (B, H)),
+            "state_f32": (torch.float32, (B, H, d, d)),
+        }
+        present = {n for n in EXPORT_REGIONS if n != "fill" and getattr(L, n) != ABSENT}
+        if c.mode == MODE["window"]:
+            present.add("fill")
+        return {n: spec[n] for n in EXPORT_REGIONS if n in present}
+
+    def export(self, names=None, device="cpu", stream=None, check: bool = True) -> dict:
+        """Copy state regions out through lq_state_export into new tensors on
+        `device` (host tensors are pinned).  names: regions to copy (None = all
+        this state keeps).  Synchronizes the stream.  Raises LQError when the
+        device error word is set, unless check is False."""
+        shapes = self.export_shapes()
+        names = list(shapes) if names is None else list(names)
+        dev = torch.device(device)
+        pin = dev.type == "cpu" and torch.cuda.is_available()
+        out, dst = {}, Export()
+        for n in names:
+            if n not in shapes:
+                raise KeyError(f"this state keeps no {n}")
+            dt, shape = shapes[n]
+            x = torch.empty(shape, dtype=dt, device=dev, pin_memory=pin)
+            out[n] = x
+            if x.numel():
+                setattr(dst, n, x.data_ptr())
+        st = lib().lq_state_export(self._h, ctypes.byref(dst), _stream_ptr(stream, self.device))
+        if st != LQ_OK and (check or st in (LQ_ERR_INVALID_ARG, LQ_ERR_STATE, LQ_ERR_CUDA)):
+            raise LQError(st, "lq_state_export")
+        return out
+
+    def read(self, name: str, device="cpu", check: bool = True) -> torch.Tensor:
+        """One region of the state, copied out through lq_state_export."""
+        return self.export([name], device=device, check=check)[name]
 
     def device_status(self, stream=None) -> int:
         """Synchronize and return the status of the device error word (LQ_OK if clean)."""
@@ -295,7 +359,9 @@ class DecodeState:
 
     # ------------------------------------------------------------ inspection
     def view(self, name: str) -> torch.Tensor | None:
-        """A tensor view of one workspace region (see lq_layout in include/lq.h)."""
+        """A writable tensor view of one workspace region, laid out as lq_layout
+        says (internal layout: read the state with export(); this is for
+        writing a state in, as a checkpoint restore does)."""
         L, c = self.layout, self.cfg
         off = getattr(L, name)
         if off == ABSENT:

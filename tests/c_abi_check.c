@@ -3,7 +3,8 @@
  * headers: the header compiles as C, the library links, and the host-only
  * calls behave as declared -- workspace sizing and layout, config
  * validation, create / destroy, the host-side refusals of calls made out of
- * order or with bad pointers, resume validation and the error text.  No call
+ * order or with bad pointers, the export's argument checks, resume
+ * validation and the error text.  No call
  * here launches a kernel or touches a device pointer (create only records
  * the workspace address), so it runs on a machine without a GPU.
  * Exit status 0 when every check holds; otherwise the failing line.
@@ -84,6 +85,18 @@ int main(void) {
     CHECK(lq_decode_step(h, NULL, p, p, pf, pf, po, NULL) == LQ_ERR_INVALID_ARG);
     CHECK(lq_decode_step(h, (const void *)((uintptr_t)p + 8), p, p, pf, pf, po, NULL) == LQ_ERR_INVALID_ARG);
     CHECK(lq_decode_step_active(h, p, p, p, pf, pf, NULL, po, NULL) == LQ_ERR_STATE);   /* not ragged */
+
+    /* export: a NULL destination set, a region the mode lacks and a call
+     * before the prefill are refused on the host, before any copy */
+    lq_export ex;
+    memset(&ex, 0, sizeof(ex));
+    CHECK(lq_state_export(NULL, &ex, NULL) == LQ_ERR_INVALID_ARG);
+    CHECK(lq_state_export(h, NULL, NULL) == LQ_ERR_INVALID_ARG);
+    ex.state_f32 = po;                                 /* windowed handles keep no FP32 state */
+    CHECK(lq_state_export(h, &ex, NULL) == LQ_ERR_INVALID_ARG);
+    ex.state_f32 = NULL;
+    ex.codes = (int8_t *)po;
+    CHECK(lq_state_export(h, &ex, NULL) == LQ_ERR_STATE);
 
     /* resume: the shared phase may hold 0..W buffered tokens */
     CHECK(lq_state_resume(h, -1) == LQ_ERR_INVALID_ARG);

@@ -31,11 +31,12 @@ def unit_inputs(tb: inputs.TokenBatch, units) -> tuple:
 
 
 def snapshot(st: lq.DecodeState) -> dict:
-    out = {}
-    for name in ("codes", "row_scale", "col_smooth", "comp_index", "comp_row_vec", "comp_col_vec"):
-        v = st.view(name)
-        out[name] = None if v is None else v.detach().cpu().clone()
-    return out
+    """The encoded window-start state, read through lq_state_export (absent
+    regions are None)."""
+    names = ("codes", "row_scale", "col_smooth", "comp_index", "comp_row_vec", "comp_col_vec")
+    shapes = st.export_shapes()
+    got = st.export([n for n in names if n in shapes])
+    return {n: got.get(n) for n in names}
 
 
 def to_device(tb: inputs.TokenBatch, device) -> inputs.TokenBatch:
@@ -91,7 +92,7 @@ def import_encoded(st: lq.DecodeState, ref: oracle.RunResult, f: int, units=None
 
     put("codes", ref.Q[:, f])
     put("row_scale", ref.sigma[:, f])
-    if st.view("col_smooth") is not None:
+    if "col_smooth" in st.export_shapes():
         put("col_smooth", ref.s[:, f])
     nr, nc = st.cfg.n_comp_rows, st.cfg.n_comp_cols
     if st.cfg.mode == 0 and nr + nc > 0:

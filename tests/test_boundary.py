@@ -14,7 +14,8 @@ def test_exports_every_declared_symbol():
                           "lq_prefill_state", "lq_decode_step", "lq_window_flush", "lq_window_fill",
                           "lq_device_status", "lq_state_destroy", "lq_last_error_string",
                           "lq_decode_step_active", "lq_window_flush_pending", "lq_prefill_sequences",
-                          "lq_prefill_tokens", "lq_prefill_sequences_tokens", "lq_state_resume"}
+                          "lq_prefill_tokens", "lq_prefill_sequences_tokens", "lq_state_resume",
+                          "lq_state_export"}
     L = lq.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -202,3 +203,37 @@ def test_resume_validates_on_the_host():
             assert L.lq_window_fill(h) == 5
         assert L.lq_state_destroy(h) == lq.LQ_OK
     assert L.lq_state_resume(None, 0) == lq.LQ_ERR_INVALID_ARG
+
+
+def test_export_struct_matches_the_header():
+    """The binding's lq_export fields are the header's, in the header's order."""
+    import re
+    with open(lq.HEADER) as f:
+        text = f.read()
+    body = re.search(r"typedef struct lq_export \{(.*?)\} lq_export;", text, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"\*\s*(\w+)\s*;", body)
+    assert fields == [n for n, _ in lq.Export._fields_]
+    assert ctypes.sizeof(lq.Export) == 8 * len(fields)
+
+
+def test_export_refusals_without_a_gpu():
+    """lq_state_export validates on the host before any copy: a bad handle, a
+    NULL destination set, a region the mode lacks, a call before the prefill."""
+    L = lq.lib()
+    assert L.lq_state_export(None, ctypes.byref(lq.Export()), None) == lq.LQ_ERR_INVALID_ARG
+    cfg = lq.make_config(2, 3, 64, window=8)
+    n = lq.workspace_bytes(cfg)
+    h = ctypes.c_void_p()
+    assert L.lq_state_create(ctypes.byref(cfg), ctypes.c_void_p(1 << 20), n, ctypes.byref(h)) == lq.LQ_OK
+    try:
+        assert L.lq_state_export(h, None, None) == lq.LQ_ERR_INVALID_ARG
+        dst = lq.Export()
+        dst.state_f32 = 1 << 21                      # windowed handles keep no FP32 state
+        assert L.lq_state_export(h, ctypes.byref(dst), None) == lq.LQ_ERR_INVALID_ARG
+        assert "state_f32" in lq.last_error()
+        dst = lq.Export()
+        dst.codes = 1 << 21
+        assert L.lq_state_export(h, ctypes.byref(dst), None) == lq.LQ_ERR_STATE   # before any prefill
+    finally:
+        L.lq_state_destroy(h)

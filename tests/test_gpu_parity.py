@@ -80,11 +80,12 @@ def test_naive_prefill_bit_exact(d):
     st = lq.DecodeState(B, H, d, mode="naive", device=DEV)
     st.prefill(S0.to(DEV).contiguous())
     p = oracle_params(d, nr=0, nc=0, smooth=0, mode="naive")
+    got = st.export(["codes", "row_scale"])
     for u in range(B * H):
         b, h = divmod(u, H)
         e = oracle.encode(p, S0[b, h].double().numpy())
-        np.testing.assert_array_equal(st.view("codes")[b, h].cpu().numpy(), e.Q)
-        np.testing.assert_array_equal(st.view("row_scale")[b, h].cpu().numpy(), e.sigma)
+        np.testing.assert_array_equal(got["codes"][b, h].numpy(), e.Q)
+        np.testing.assert_array_equal(got["row_scale"][b, h].numpy(), e.sigma)
 
 
 # ------------------------------------------------------------ windowed decode
@@ -164,6 +165,14 @@ def test_window_decode_variants(d, gate, W, nr, nc):
     _window_case(d, gate, torch.bfloat16, W, nr, nc, B, H, T, seed=11 + W, S0_kind="normal")
 
 
+@pytest.mark.parametrize("W", [128, 256])
+def test_window_decode_long_gdn_windows(W):
+    """The sweep's longest windows (GDN, d = 128, bf16 inputs, 2 + 2
+    compensators): two full windows and half of a third, every window
+    teacher-forced from the oracle's encoding."""
+    _window_case(128, "scalar", torch.bfloat16, W, 2, 2, 2, 3, 2 * W + W // 2 + 1, seed=13 + W, S0_kind="normal")
+
+
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("gate", ["scalar", "channel"])
 def test_window_decode_fp32_inputs(d, gate):
@@ -228,7 +237,7 @@ def test_fp32_state_decode(d, gate, dtype):
                      *unit_inputs(tb, range(B * H)))
     o_ref = ref.o.reshape(B, H, T, d).transpose(2, 0, 1, 3)
     assert rel_l2(o_gpu.numpy(), o_ref) <= 1e-5
-    S_gpu = st.view("state_f32").reshape(-1, d, d).cpu().numpy()
+    S_gpu = st.read("state_f32").reshape(-1, d, d).numpy()
     assert rel_l2(S_gpu, ref.S_final) <= 1e-5
 
 
@@ -251,5 +260,5 @@ def test_naive_int8_decode(d, gate):
         import_encoded(st, ref, t)
         o_t = st.decode_step(tbd.q[t], tbd.k[t], tbd.v[t], tbd.g[t], tbd.beta[t])
         assert rel_l2(o_t.cpu().numpy(), o_ref[t]) <= 1e-5, t
-        frac, worst = compare_codes(st.view("codes").reshape(-1, d, d).cpu().numpy(), ref.Q[:, t + 1])
+        frac, worst = compare_codes(st.read("codes").reshape(-1, d, d).numpy(), ref.Q[:, t + 1])
         assert frac >= 0.999 and worst <= 1, (t, frac, worst)

@@ -152,7 +152,7 @@ def test_ragged_without_masks_matches_shared_phase(gate):
     assert rag.device_status() == lq.LQ_OK and ref.device_status() == lq.LQ_OK
     assert torch.equal(o_rag, o_ref)
     for name in ("codes", "row_scale", "col_smooth", "comp_index", "buf_delta"):
-        assert torch.equal(rag.view(name), ref.view(name)), name
+        assert torch.equal(rag.read(name), ref.read(name)), name
     assert (rag.fills() == T % W).all()
 
 
