@@ -262,3 +262,35 @@ def test_naive_int8_decode(d, gate):
         assert rel_l2(o_t.cpu().numpy(), o_ref[t]) <= 1e-5, t
         frac, worst = compare_codes(st.read("codes").reshape(-1, d, d).numpy(), ref.Q[:, t + 1])
         assert frac >= 0.999 and worst <= 1, (t, frac, worst)
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_naive_int8_decode_many_units_per_cta(gate, dtype):
+    """The naive kernel is persistent: with 38 x 32 units every CTA walks several
+    units through its slot ring.  Sampled units are checked against the oracle,
+    free-running and teacher-forced per token."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    d, H, T = 128, 32, 6
+    B = -(-8 * sms // H) + 1
+    tb = inputs.tokens(33, 0, T, B, H, d, d, per_channel_gate=(gate == "channel"), dtype=dtype)
+    S0 = _state("normal", 33, B, H, d)
+    st = lq.DecodeState(B, H, d, gate=gate, mode="naive", in_dtype=dtype, device=DEV)
+    st.prefill(S0.to(DEV).contiguous())
+    o_gpu, _ = gpu_run(st, to_device(tb, DEV))
+    assert st.device_status() == lq.LQ_OK
+    units = sorted(np.random.default_rng(33).choice(B * H, 8, replace=False).tolist())
+    ref = oracle.run(oracle_params(d, gate=gate, mode="naive"), S0.reshape(-1, d, d)[units].double().numpy(),
+                     *unit_inputs(tb, units))
+    o_s = o_gpu.reshape(T, B * H, d)[:, units].transpose(0, 1).numpy()
+    assert rel_l2(o_s, ref.o) <= 1e-3
+    tbd = to_device(tb, DEV)
+    st.prefill(S0.to(DEV).contiguous())
+    for t in range(T):
+        import_encoded(st, ref, t, units)
+        o_t = st.decode_step(tbd.q[t], tbd.k[t], tbd.v[t], tbd.g[t], tbd.beta[t])
+        got = o_t.reshape(B * H, d)[units].cpu().numpy()
+        assert rel_l2(got, ref.o[:, t]) <= 1e-5, t
+        codes = st.read("codes").reshape(B * H, d, d)[units].numpy()
+        frac, worst = compare_codes(codes, ref.Q[:, t + 1])
+        assert frac >= 0.999 and worst <= 1, (t, frac, worst)
