@@ -102,8 +102,12 @@ enum {
 enum { LQ_SELECT_L2 = 0, LQ_SELECT_MAXABS = 1 };
 enum { LQ_DTYPE_F32 = 0, LQ_DTYPE_BF16 = 1 };
 
-/* Device error codes in the workspace error word (lq_layout.err, int32[0]). */
-enum { LQ_DEVERR_NONE = 0, LQ_DEVERR_RANGE = 1, LQ_DEVERR_TIMEOUT = 2, LQ_DEVERR_WINDOW_FULL = 3 };
+/* Device error codes in the workspace error word (lq_layout.err, int32[0]).
+ * LQ_DEVERR_BOUNDS is raised only by the bounds-checked build of the library
+ * (liblq_checked.so): a computed index outside its region, whose access was
+ * skipped; lq_device_status() reports it as LQ_ERR_DEVICE. */
+enum { LQ_DEVERR_NONE = 0, LQ_DEVERR_RANGE = 1, LQ_DEVERR_TIMEOUT = 2, LQ_DEVERR_WINDOW_FULL = 3,
+       LQ_DEVERR_BOUNDS = 4 };
 
 typedef struct lq_config {
     int32_t batch;        /* sequences, >= 1                                     */

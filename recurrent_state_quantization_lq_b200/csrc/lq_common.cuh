@@ -90,6 +90,28 @@ __device__ __forceinline__ void report_error(int32_t *err, int code, int unit, i
     }
 }
 
+// ------------------------------------------------------ bounds-checked build
+//
+// Built with -DLQ_BOUNDS_CHECK (liblq_checked.so), the kernels test the
+// indices they compute from workspace contents or launch arguments before
+// they use them; an index outside its region is recorded as LQ_DEVERR_BOUNDS
+// (unit, detail) and the access is skipped.  The normal build compiles every
+// check away.
+#ifdef LQ_BOUNDS_CHECK
+constexpr bool kBoundsChecked = true;
+#else
+constexpr bool kBoundsChecked = false;
+#endif
+
+// True when lo <= idx < hi; in the checked build a violation is also reported.
+__device__ __forceinline__ bool in_bounds(int32_t *err, long long idx, long long lo, long long hi, int unit,
+                                          int detail) {
+    if (!kBoundsChecked) return true;
+    if (idx >= lo && idx < hi) return true;
+    report_error(err, LQ_DEVERR_BOUNDS, unit, detail);
+    return false;
+}
+
 // ------------------------------------------------- mbarrier + bulk async copies
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

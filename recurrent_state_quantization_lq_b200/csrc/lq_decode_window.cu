@@ -177,6 +177,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 report_error(w.err, LQ_DEVERR_WINDOW_FULL, u, n_buf);
                 continue;
             }
+            // checked build: a negative count (a corrupted workspace) is skipped too
+            if (RAGGED && !in_bounds(w.err, n_buf, 0, w.window, u, -10)) continue;
             const int nchunks = (n_buf + E - 1) / E;
             unsigned char *dst = acquire(u, -1);
             if (dst == nullptr) { drain(); return; }
@@ -268,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             beta_n = a.beta[un];
             if (!KDA) { g_n = a.g[un]; G_n = w.gate_sum[un]; }
         }
-        if (RAGGED && (!active || n_buf >= w.window)) {   // not decoded this step (nor loaded)
+        if (RAGGED && (!active || n_buf >= w.window || (kBoundsChecked && n_buf < 0))) {   // not decoded (nor loaded)
             if (!KDA && un < units) {
                 G_n = G_n + (double)g_n;
                 gam_n = exp_of_double(G_n);
@@ -580,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
 
         // ------------------------------------------------ A4: emit and append
-        if (owns_row) {
+        if (owns_row && in_bounds(w.err, n_buf, 0, w.window, u, -12)) {
             const int i = tid;
             // sigma_i times the INT8 products, rounded before the sum as a product of its own
             const float pk = Sh::TC ? p8k : sB[i], pq = Sh::TC ? p8q : sA[i];

@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
     const int units = w.units, n_buf = a.n_buf;      // one window phase for every unit
     const int nchunks = (n_buf + E - 1) / E;
     const FlushMeta M = flush_meta_layout<D, KDA>(ncr, ncc, cis);
+    if (!in_bounds(w.err, n_buf, 0, w.window + 1, -1, -20)) return;   // checked build; every thread alike
 
     extern __shared__ __align__(128) unsigned char sm[];
     uint64_t *full = reinterpret_cast<uint64_t *>(sm);

@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(kThreads) flush_split_kernel(EncodeArgs a) {
         // ------------------------------------ which candidates are due
         const int k = p0 + tid;
         const int n = (k < per) ? a.fill[cid + k * ncl] : 0;
+        if (k < per) in_bounds(w.err, n, 0, (long long)w.window + 1, cid + k * ncl, -30);   // checked build: report
         const bool due = (k < per) && n >= a.flush_min;
         const uint32_t mask = __ballot_sync(0xffffffffu, due);
         if (lane == 0) ballots[warp] = mask;

@@ -117,6 +117,8 @@ __global__ void __launch_bounds__(kTile, 2) prefill_tokens_kernel(TokenPrefillAr
     const int lane0 = lane - cg;                                     // the row block's first lane
     const int units = a.w.units, b = u / a.heads;
     if (a.seq_mask != nullptr && a.seq_mask[b] == 0) return;       // sequence not restarted
+    if (a.lengths != nullptr && threadIdx.x == 0)   // checked build: report a length outside 0..n_tokens
+        in_bounds(a.w.err, a.lengths[b], 0, (long long)a.n_tokens + 1, u, -40);
     const int T = a.lengths != nullptr ? min(max(a.lengths[b], 0), a.n_tokens) : a.n_tokens;
     auto col = [&](int m) { return m * 4 * LPR + cg * 4; };          // first of 4 owned columns in piece m
     // after the butterfly this lane holds the sum of row r0 + mine

@@ -14,7 +14,9 @@ import re
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblq.so")
+# LQ_LIBRARY may name another build of the same C ABI, e.g. the bounds-checked
+# liblq_checked.so (python -m recurrent_state_quantization_lq_b200.build --bounds-check)
+LIB_PATH = os.environ.get("LQ_LIBRARY") or os.path.join(_HERE, "liblq.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "lq.h")
 
 # enums of include/lq.h
@@ -25,6 +27,8 @@ MODE = {"window": 0, "naive": 1, "fp32": 2}
 SELECT = {"l2": 0, "maxabs": 1}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 ABSENT = ctypes.c_size_t(-1).value
+
+LQ_DEVERR_BOUNDS = 4   # device error code of the bounds-checked build
 
 STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED", 3: "LQ_ERR_WORKSPACE",
                 4: "LQ_ERR_WINDOW_FULL", 5: "LQ_ERR_RANGE", 6: "LQ_ERR_CUDA", 7: "LQ_ERR_DEVICE",

@@ -237,3 +237,16 @@ def test_export_refusals_without_a_gpu():
         assert L.lq_state_export(h, ctypes.byref(dst), None) == lq.LQ_ERR_STATE   # before any prefill
     finally:
         L.lq_state_destroy(h)
+
+
+def test_checked_build_exports_every_declared_symbol():
+    """The bounds-checked variant (built by __graft_entry__.build() and
+    `python -m recurrent_state_quantization_lq_b200.build --bounds-check`)
+    exports the same C ABI."""
+    import os
+    from recurrent_state_quantization_lq_b200 import build as lqbuild
+    if not os.path.exists(lqbuild.LIB_CHECKED):
+        pytest.skip("liblq_checked.so not built")
+    L = ctypes.CDLL(lqbuild.LIB_CHECKED)
+    for n in lq.header_symbols():
+        assert hasattr(L, n), n
