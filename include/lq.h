@@ -47,6 +47,15 @@
  *  - Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  All
  *    device work is enqueued on it, asynchronously; no call synchronizes except
  *    lq_device_status() and lq_state_export().
+ *  - Overlapped launches.  The windowed decode kernel is launched as a
+ *    programmatic dependent of the kernel before it in the stream: its CTAs
+ *    set up while that kernel finishes, and read the step's inputs and the
+ *    window buffer only after it has completed.  When the handle's previous
+ *    call that enqueued device work was also a decode, a CTA fetches its
+ *    first INT8 code tile before that point too; the workspace's codes must
+ *    therefore not be written by any means but this library's calls.  A
+ *    caller that writes the encoded state itself (a checkpoint restore) calls
+ *    lq_state_resume() afterwards: the decode after it fetches nothing early.
  *  - Errors.  Every call returns an lq_status.  Errors found on the host are
  *    returned at once and leave the state untouched; the text of the last one
  *    on the calling thread is lq_last_error_string().  Errors found on the
@@ -317,7 +326,9 @@ LQ_API lq_status lq_prefill_sequences_tokens(lq_handle h, const float *d_S0, con
  * the noted count.  n_buf: tokens buffered in the shared window, 0..W
  * (windowed mode), 0 in the other modes; a ragged handle takes its counts
  * from the workspace and ignores n_buf (pass 0).  No device work; the next
- * decode, flush or prefill continues exactly where the checkpoint stood.
+ * decode, flush or prefill continues exactly where the checkpoint stood, and
+ * the next decode reads the codes only after the kernel before it in its
+ * stream has completed.
  * Errors: LQ_ERR_INVALID_ARG for a bad handle or an n_buf out of range.
  * Source: none (checkpointing).
  */

@@ -116,6 +116,9 @@ struct lq_state_s {
     int32_t n_buf;
     int prefilled;
     int codes_map_ready;
+    // No call but a decode was made since the codes were last written: the
+    // previous kernel in any stream order can no longer be their writer.
+    int codes_settled;
     // ragged handles: every unit is known to be in the same window phase
     // (n_buf tokens) until an active mask or a sequence restart is used
     int aligned;
@@ -204,6 +207,7 @@ lq_status lq_state_create(const lq_config *cfg, void *d_workspace, size_t bytes,
     h->prefilled = 0;
     h->aligned = 0;
     h->codes_map_ready = 0;
+    h->codes_settled = 0;
     *out = h;
     return LQ_OK;
 }
@@ -217,6 +221,7 @@ lq_status lq_state_destroy(lq_handle h) {
 
 lq_status lq_state_resume(lq_handle h, int32_t n_buf) {
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    h->codes_settled = 0;
     const lq_config &c = h->cfg;
     const int32_t max_buf = (c.mode == LQ_MODE_WINDOW && !c.ragged) ? c.window : 0;
     if (n_buf < 0 || n_buf > max_buf) return fail(LQ_ERR_INVALID_ARG, "n_buf out of range for this handle");
@@ -234,6 +239,7 @@ int32_t lq_window_fill(lq_handle h) {
 lq_status lq_prefill_state(lq_handle h, const float *d_S0, void *stream) {
     Range nvtx_range("lq_prefill_state");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    h->codes_settled = 0;
     if (d_S0 != nullptr && !aligned(d_S0, 16)) return fail(LQ_ERR_INVALID_ARG, "S0 must be 16-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const lq_config &c = h->cfg;
@@ -277,6 +283,7 @@ lq_status lq_prefill_tokens(lq_handle h, const float *d_S0, const void *d_q, con
                             const float *d_g, const float *d_beta, int32_t n_tokens, float *d_o, void *stream) {
     Range nvtx_range("lq_prefill_tokens");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    h->codes_settled = 0;
     if (n_tokens < 0) return fail(LQ_ERR_INVALID_ARG, "negative n_tokens");
     if (n_tokens == 0) return lq_prefill_state(h, d_S0, stream);
     const lq_config &c = h->cfg;
@@ -322,6 +329,7 @@ lq_status lq_prefill_sequences_tokens(lq_handle h, const float *d_S0, const void
                                       const int32_t *d_lengths, const uint8_t *d_mask, float *d_o, void *stream) {
     Range nvtx_range("lq_prefill_sequences_tokens");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    h->codes_settled = 0;
     const lq_config &c = h->cfg;
     if (!c.ragged) return fail(LQ_ERR_STATE, "lq_prefill_sequences_tokens needs a ragged handle");
     if (!h->prefilled) return fail(LQ_ERR_STATE, "lq_prefill_sequences_tokens before lq_prefill_state");
@@ -383,12 +391,14 @@ lq_status decode_impl(lq_handle h, const void *d_q, const void *d_k, const void 
     a.fill = c.ragged ? reinterpret_cast<int32_t *>(h->ws + h->lay.fill) : nullptr;
     a.active = c.ragged ? d_active : nullptr;
     a.heads = c.heads;
+    a.codes_settled = h->codes_settled;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (c.mode == LQ_MODE_WINDOW) e = lq::launch_decode_window(a, c.d_k, c.gate, c.in_dtype, s);
     else if (c.mode == LQ_MODE_NAIVE) e = lq::launch_decode_naive(a, c.d_k, c.gate, c.in_dtype, s);
     else e = lq::launch_decode_fp32(a, c.d_k, c.gate, c.in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "launching the decode kernel");
+    h->codes_settled = 1;
     if (c.mode == LQ_MODE_WINDOW && !c.ragged) h->n_buf += 1;
     if (c.ragged) {
         if (d_active != nullptr) h->aligned = 0;
@@ -401,6 +411,7 @@ lq_status decode_impl(lq_handle h, const void *d_q, const void *d_k, const void 
 // least flush_min buffered tokens (ragged phases).
 lq_status flush_impl(lq_handle h, int flush_min, void *stream) {
     const lq_config &c = h->cfg;
+    h->codes_settled = 0;
     if (c.mode != LQ_MODE_WINDOW) return LQ_OK;
     if (!h->prefilled) return fail(LQ_ERR_STATE, "flush before lq_prefill_state");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -464,6 +475,7 @@ lq_status lq_window_flush_pending(lq_handle h, void *stream) {
 lq_status lq_prefill_sequences(lq_handle h, const float *d_S0, const uint8_t *d_mask, void *stream) {
     Range nvtx_range("lq_prefill_sequences");
     if (!check_handle(h)) return fail(LQ_ERR_INVALID_ARG, "invalid handle");
+    h->codes_settled = 0;
     const lq_config &c = h->cfg;
     if (!c.ragged) return fail(LQ_ERR_STATE, "lq_prefill_sequences needs a ragged handle");
     if (!h->prefilled) return fail(LQ_ERR_STATE, "lq_prefill_sequences before lq_prefill_state");

@@ -186,6 +186,23 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return p;
 }
 
+// --------------------------------------------- programmatic dependent launch
+//
+// A kernel launched with programmatic stream serialization may start while the
+// kernel before it in the stream is still running.  It must not read anything
+// that kernel may write, nor write anything it may read, before
+// grid_dependency_wait() returns in the thread that makes the access; the
+// wait returns once the earlier kernel has completed and its writes are
+// visible (immediately, when the launch had no such attribute).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel in the stream start once every CTA of this grid has
+// signalled (or exited).  Signalled only after this CTA's own wait, so that a
+// kernel which starts early finds everything before its predecessor completed.
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // About one second at the B200's clocks: a bulk copy that has not landed by
 // then never will.
 constexpr long long kWaitBudgetCycles = 2000000000LL;

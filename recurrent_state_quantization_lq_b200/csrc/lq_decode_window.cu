@@ -170,6 +170,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             for (int i = 0; i < kSlots; ++i)
                 if (armed & (1u << i)) mbar_wait(&full[i], i < slot ? ph : (ph ^ 1u), kWaitBudgetCycles);
         };
+        // The first unit's code tile takes ring slot 1 of the first round, as the
+        // loop below would give it.  With the codes settled it is fetched before
+        // the wait for the previous kernel in the stream, which cannot write it.
+        const int early_u = (!RAGGED && a.codes_settled && blockIdx.x < units) ? (int)blockIdx.x : -1;
+        if (early_u >= 0) {
+            armed |= 2u;                           // slot 1's empty barrier is in its first phase
+            mbar_arrive_expect_tx(&full[1], D * D);
+            tma_load_2d(ring + kSlotBytes, &codes_map, 0, early_u * D, &full[1]);
+        }
+        grid_dependency_wait();
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
             const int n_buf = unit_fill(u);
             if (!unit_active(u)) continue;
@@ -199,11 +209,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 if (ncc > 0) bulk_g2s(dst + M.ccol, w.comp_col_vec + (size_t)u * ncc * D, 4 * D * ncc, bar);
             }
             advance();
-            dst = acquire(u, -2);
-            if (dst == nullptr) { drain(); return; }
-            bar = &full[slot];
-            mbar_arrive_expect_tx(bar, D * D);
-            tma_load_2d(dst, &codes_map, 0, u * D, bar);
+            if (u != early_u) {
+                dst = acquire(u, -2);
+                if (dst == nullptr) { drain(); return; }
+                bar = &full[slot];
+                mbar_arrive_expect_tx(bar, D * D);
+                tma_load_2d(dst, &codes_map, 0, u * D, bar);
+            }
             advance();
             for (int c = 0; c < nchunks; ++c) {
                 dst = acquire(u, -3 - c);
@@ -242,6 +254,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const uint32_t tmem = Sh::TC ? *tmem_slot : 0u;   // lane i = state row i
     uint32_t mph = 0;                                 // phase of the tcgen05 pass barrier
     bool tc_inflight = false;                         // a pass was issued and not yet seen complete
+    grid_dependency_wait();                           // the inputs and the buffer may still be in writing
+    if (tid == 0) grid_dependents_launch();
     int u = blockIdx.x;
     float beta_n = 0.0f, g_n = 0.0f, gam_n = 0.0f;
     double G_n = 0.0;
@@ -635,9 +649,19 @@ cudaError_t launch_r(const DecodeArgs &a, cudaStream_t s) {
     // inside a stream capture make no attribute calls.
     const cudaError_t e = opt_in_smem<decode_window_kernel<D, KDA, InT, KeyT, RAGGED, TCP>>(Sh::SMEM);
     if (e != cudaSuccess) return e;
-    const int grid = min(a.w.units, kCtasPerSm * sm_count());
-    kern<<<grid, kThreads, Sh::SMEM, s>>>(a, *reinterpret_cast<const CUtensorMap *>(a.codes_map));
-    return cudaGetLastError();
+    // A programmatic dependent of the previous kernel in the stream: the CTAs
+    // set up (barriers, tensor memory, the first code tile) while it finishes.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(min(a.w.units, kCtasPerSm * sm_count()));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Sh::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, *reinterpret_cast<const CUtensorMap *>(a.codes_map));
 }
 
 // Shared window phases compile without the per-unit counts and the active mask.

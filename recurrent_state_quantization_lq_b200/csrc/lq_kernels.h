@@ -103,6 +103,10 @@ struct DecodeArgs {
     int32_t *fill;
     const uint8_t *active;
     int heads;         // units per sequence
+    // The INT8 codes were last written before the kernel that precedes this
+    // launch in its stream: the first code tile may be fetched before that
+    // kernel completes (shared window phases only).
+    int codes_settled;
 };
 
 struct TokenPrefillArgs {
