@@ -143,7 +143,8 @@ typedef struct lq_config {
 #define LQ_ABSENT ((size_t)-1)
 typedef struct lq_layout {
     size_t total_bytes;
-    size_t err;           /* int32[64]: [0] LQ_DEVERR_*, [1] unit, [2] detail     */
+    size_t err;           /* int32[64]: [0] LQ_DEVERR_*, [1] unit, [2] detail;
+                             [32..33] the windowed decode's unit-ticket counter */
     size_t codes;         /* int8  [N][d_v][d_k]                 window, naive    */
     size_t row_scale;     /* f32   [N][d_v]       sigma          window, naive    */
     size_t col_smooth;    /* f32   [N][d_k]       s              window           */

@@ -17,15 +17,19 @@
 // buffer.  It writes no state.
 //
 // Persistent and warp-specialized: four CTAs per SM walk the (sequence, head)
-// units.  In each CTA one producer thread streams every unit's data through a
-// ring of three 16 KB shared-memory slots -- a meta segment (row scales,
-// smoothing factors, q/k/v, gate, compensators) by 1-D bulk async copies, the
-// INT8 tile by a 2-D tensor copy with 128-byte swizzle, then the buffered
-// entries in chunks of up to 16 -- and four consumer warps compute.  Each
-// slot has a full mbarrier (bytes landed) and an empty mbarrier that every
-// consumer thread arrives on after its last read, so no block-wide barrier is
-// spent on releasing slots; the consumers meet at one barrier after the
-// operand prep and one per chunk.  Each thread keeps its row scale sigma_i in a
+// units in whole rounds (CTA b takes b, b + grid, ...), and the units of the
+// last, partial round go to the CTAs that get there first, by a ticket
+// counter.  In each CTA one producer thread loads a unit's scalars (beta, the
+// scalar gate) and streams its data through a ring of three 16 KB
+// shared-memory slots -- a meta segment (row scales, smoothing factors,
+// q/k/v, gate, compensators) by 1-D bulk async copies, the INT8 tile by a 2-D
+// tensor copy with 128-byte swizzle, then the buffered entries in chunks of up
+// to 16 -- and four consumer warps compute.  Each slot has a full mbarrier
+// (bytes landed, and for a meta segment the producer's record of the unit) and
+// an empty mbarrier that every consumer thread arrives on after its last read,
+// so no block-wide barrier is spent on releasing slots; the consumers meet at
+// one barrier when a unit's record arrives, one after the operand prep and one
+// per chunk.  Each thread keeps its row scale sigma_i in a
 // register, so the meta slot goes back before the INT8 pass starts.
 //
 // The INT8 pass is an exact integer dot product on the tensor cores.  Each
@@ -67,6 +71,20 @@ using namespace dec;
 
 __device__ __forceinline__ bool consumer_sync_or(bool pred) { return named_sync_or(kConsumerBarrier, kConsumers, pred); }
 
+// What the producer tells the consumers about the unit whose meta segment
+// fills a slot (u < 0: no unit is left).  Scalar gate: G_t = G_{t-1} + g_t and
+// gamma_t = exp(G_t).
+struct UnitRec {
+    double G;
+    float gam;
+    float beta;
+    int u;
+    int n_buf;
+};
+
+// The unit-ticket counter: a 64-bit word in the error region (int32 index).
+constexpr int kTicketWord = 32;
+
 template <int D, bool KDA, typename InT, typename KeyT, bool TCP>
 struct Shape {
     static constexpr int KB = (int)sizeof(KeyT);
@@ -88,8 +106,9 @@ struct Shape {
     static constexpr int S_B8 = 0, S_EXP = S_B8 + (TC ? 4 * D : 2 * D), S_XQ = S_EXP + 8, S_XK = S_XQ + D, S_QR = S_XK + D,
                          S_KR = S_QR + D, S_A = S_KR + D, S_B = S_A + D, S_CF = S_B + D,
                          S_RED = S_CF + 64, S_FLOATS = S_RED + kConsumerWarps * RED;
-    static constexpr int OFF_BARS = 4 * S_FLOATS;                  // then the ring, 1024-aligned
-    static constexpr int OFF_RING = align_up(OFF_BARS + 16 * kSlots + 16, 1024);   // + MMA barrier, TMEM slot
+    static constexpr int OFF_BARS = 4 * S_FLOATS;                  // then the unit records, the ring (1024-aligned)
+    static constexpr int OFF_REC = OFF_BARS + 16 * kSlots + 16;    // + MMA barrier, TMEM slot
+    static constexpr int OFF_RING = align_up(OFF_REC + (int)sizeof(UnitRec) * kSlots, 1024);
     static constexpr int SMEM = OFF_RING + kSlots * kSlotBytes + 1024;   // + alignment slack
     static_assert(E >= 4 && E <= kPer * kConsumerWarps, "chunk size");
     static_assert(MT >= 1, "m-tiles");
@@ -119,6 +138,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     uint64_t *empty = full + kSlots;
     uint64_t *mma_bar = empty + kSlots;            // tcgen05 pass complete (d = 128)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + 1);
+    UnitRec *rec = reinterpret_cast<UnitRec *>(sm + Sh::OFF_REC);   // one per ring slot
     unsigned char *ring = sm + Sh::OFF_RING;
     unsigned char *dig = sm + Sh::S_B8 * 4;        // digit operand (scratch starts at sm)
 
@@ -147,12 +167,63 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (warp == kConsumerWarps) {
         if (lane != 0) return;
         const uint32_t in_b = (uint32_t)sizeof(InT) * D;
+        // Units: CTA b walks b, b + grid, ... through the whole rounds; the
+        // units of the last, partial round are handed out by a ticket counter
+        // in the workspace to the CTAs that get there first.  A launch then
+        // draws n_dyn + grid tickets (one per such unit, and one per CTA that
+        // finds none left), and launches of a state never draw at the same time
+        // (each draws only after the kernel before it has completed), so one
+        // launch's tickets are consecutive counter values: t mod (n_dyn + grid)
+        // runs over each value once, whatever the counter started from.
+        const int grid = (int)gridDim.x;
+        const int rounds = units / grid;
+        const int n_dyn = units - rounds * grid;
+        const unsigned long long n_tk = (unsigned long long)(n_dyn + grid);
+        unsigned long long *tickets = reinterpret_cast<unsigned long long *>(w.err + kTicketWord);
+        struct Scalars {
+            int n;
+            bool act;
+            float beta, g;
+            double gs;
+        };
+        auto fetch = [&](int uu, Scalars &s) {   // loads left in flight until the values are used
+            s.n = unit_fill(uu);
+            s.act = unit_active(uu);
+            s.beta = a.beta[uu];
+            if (!KDA) {
+                s.g = a.g[uu];
+                s.gs = w.gate_sum[uu];
+            }
+        };
+        int u = (int)blockIdx.x;
+        Scalars cur{};                             // unit u's
         int slot = 0;
         uint32_t ph = 0;
         uint32_t armed = 0;                        // slots filled at least once
-        auto acquire = [&](int u, int detail) -> unsigned char * {
+        // The record of unit u's meta slot goes out with the slot's arrival,
+        // once the unit's INT8 tile is on its way.
+        int pend = -1;
+        auto publish = [&]() {
+            UnitRec &r = rec[pend];
+            r.u = u;
+            r.n_buf = cur.n;
+            r.beta = cur.beta;
+            if (!KDA) {
+                r.G = cur.gs + (double)cur.g;
+                r.gam = exp_of_double(r.G);
+            }
+            mbar_arrive(&full[pend]);              // releases the record; the phase ends when the bytes land
+            pend = -1;
+        };
+        // a meta slot that will get no unit: it completes (once its copies have
+        // landed) as the end of the units
+        auto stop = [&](int ms) {
+            rec[ms].u = -1;
+            mbar_arrive(&full[ms]);
+        };
+        auto acquire = [&](int uu, int detail) -> unsigned char * {
             if (!mbar_wait(&empty[slot], ph ^ 1u, kWaitBudgetCycles)) {
-                report_error(w.err, LQ_DEVERR_TIMEOUT, u, detail);
+                report_error(w.err, LQ_DEVERR_TIMEOUT, uu, detail);
                 return nullptr;
             }
             armed |= 1u << slot;
@@ -161,77 +232,112 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         auto advance = [&]() {
             if (++slot == kSlots) { slot = 0; ph ^= 1u; }
         };
-        // After a timed-out acquire the consumers have stopped: wait (bounded)
-        // until every copy this thread started has landed, so that no copy
-        // still writes into the shared memory of a CTA that has exited.  Slot
-        // i was last filled in the round whose parity is ph for i < slot and
-        // ph ^ 1 for i >= slot.
-        auto drain = [&]() {
+        // After a timed-out acquire the consumers stop (a meta slot still owed a
+        // record gets the end one): wait (bounded) until every copy this thread
+        // started has landed, so that no copy still writes into the shared
+        // memory of a CTA that has exited.  Slot i was last filled in the round
+        // whose parity is ph for i < slot and ph ^ 1 for i >= slot.
+        auto fail = [&]() {
+            if (pend >= 0) stop(pend);
             for (int i = 0; i < kSlots; ++i)
                 if (armed & (1u << i)) mbar_wait(&full[i], i < slot ? ph : (ph ^ 1u), kWaitBudgetCycles);
         };
+
         // The first unit's code tile takes ring slot 1 of the first round, as the
         // loop below would give it.  With the codes settled it is fetched before
         // the wait for the previous kernel in the stream, which cannot write it.
-        const int early_u = (!RAGGED && a.codes_settled && blockIdx.x < units) ? (int)blockIdx.x : -1;
+        const int early_u = (!RAGGED && a.codes_settled) ? u : -1;
         if (early_u >= 0) {
             armed |= 2u;                           // slot 1's empty barrier is in its first phase
             mbar_arrive_expect_tx(&full[1], D * D);
             tma_load_2d(ring + kSlotBytes, &codes_map, 0, early_u * D, &full[1]);
         }
         grid_dependency_wait();
-        for (int u = blockIdx.x; u < units; u += gridDim.x) {
-            const int n_buf = unit_fill(u);
-            if (!unit_active(u)) continue;
-            if (RAGGED && n_buf >= w.window) {     // ragged phases: the window is full
-                report_error(w.err, LQ_DEVERR_WINDOW_FULL, u, n_buf);
-                continue;
+        unsigned long long tk = 0;
+        bool draw = n_dyn > 0, drawn = false;
+        fetch(u, cur);
+        for (int k = 0; u >= 0; ++k) {             // k: units walked
+            if (draw && !drawn && k == rounds - 1) {   // the ticket is back by the end of this unit
+                tk = atomicAdd(tickets, 1ull);
+                drawn = true;
             }
-            // checked build: a negative count (a corrupted workspace) is skipped too
-            if (RAGGED && !in_bounds(w.err, n_buf, 0, w.window, u, -10)) continue;
-            const int nchunks = (n_buf + E - 1) / E;
-            unsigned char *dst = acquire(u, -1);
-            if (dst == nullptr) { drain(); return; }
-            uint64_t *bar = &full[slot];
-            mbar_arrive_expect_tx(bar, (uint32_t)M.bytes);
-            bulk_g2s(dst + M.sig, w.row_scale + (size_t)u * D, 4 * D, bar);
-            bulk_g2s(dst + M.s, w.col_smooth + (size_t)u * D, 4 * D, bar);
-            bulk_g2s(dst + M.qin, reinterpret_cast<const InT *>(a.q) + (size_t)u * D, in_b, bar);
-            bulk_g2s(dst + M.kin, reinterpret_cast<const InT *>(a.k) + (size_t)u * D, in_b, bar);
-            bulk_g2s(dst + M.vin, reinterpret_cast<const InT *>(a.v) + (size_t)u * D, in_b, bar);
-            if (KDA) {
-                bulk_g2s(dst + M.gin, a.g + (size_t)u * D, 4 * D, bar);
-                bulk_g2s(dst + M.gsum, w.gate_sum + (size_t)u * D, 8 * D, bar);
+            const int n_buf = cur.n;
+            bool issue = true;
+            if (RAGGED) {
+                if (!cur.act) {
+                    issue = false;
+                } else if (n_buf >= w.window) {    // ragged phases: the window is full
+                    report_error(w.err, LQ_DEVERR_WINDOW_FULL, u, n_buf);
+                    issue = false;
+                } else if (!in_bounds(w.err, n_buf, 0, w.window, u, -10)) {
+                    issue = false;                 // checked build: a negative count (a corrupted workspace)
+                }
             }
-            if (ncomp > 0) {
-                bulk_g2s(dst + M.cidx, w.comp_index + (size_t)u * cis, 4 * cis, bar);
-                if (ncr > 0) bulk_g2s(dst + M.crow, w.comp_row_vec + (size_t)u * ncr * D, 4 * D * ncr, bar);
-                if (ncc > 0) bulk_g2s(dst + M.ccol, w.comp_col_vec + (size_t)u * ncc * D, 4 * D * ncc, bar);
-            }
-            advance();
-            if (u != early_u) {
-                dst = acquire(u, -2);
-                if (dst == nullptr) { drain(); return; }
-                bar = &full[slot];
-                mbar_arrive_expect_tx(bar, D * D);
-                tma_load_2d(dst, &codes_map, 0, u * D, bar);
-            }
-            advance();
-            for (int c = 0; c < nchunks; ++c) {
-                dst = acquire(u, -3 - c);
-                if (dst == nullptr) { drain(); return; }
-                const int e0 = c * E, ne = min(E, n_buf - e0);
-                const size_t first = (size_t)u * w.window + e0;
-                const uint32_t bd = 4u * ne * D, bk = (uint32_t)sizeof(KeyT) * ne * D;
-                const uint32_t bg = KDA ? 0u : 4u * (uint32_t)align_up(ne, 4);
-                bar = &full[slot];
-                mbar_arrive_expect_tx(bar, bd + bk + bg);
-                bulk_g2s(dst, w.buf_delta + first * D, bd, bar);
-                bulk_g2s(dst + Sh::C_KEY, reinterpret_cast<const KeyT *>(w.buf_key) + first * D, bk, bar);
-                if (!KDA) bulk_g2s(dst + Sh::C_GATE, w.buf_gate + (size_t)u * w.window_pad + e0, bg, bar);
+            if (issue) {
+                unsigned char *dst = acquire(u, -1);
+                if (dst == nullptr) { fail(); return; }
+                pend = slot;
+                uint64_t *bar = &full[slot];
+                mbar_expect_tx(bar, (uint32_t)M.bytes);   // the arrival comes with the record
+                bulk_g2s(dst + M.sig, w.row_scale + (size_t)u * D, 4 * D, bar);
+                bulk_g2s(dst + M.s, w.col_smooth + (size_t)u * D, 4 * D, bar);
+                bulk_g2s(dst + M.qin, reinterpret_cast<const InT *>(a.q) + (size_t)u * D, in_b, bar);
+                bulk_g2s(dst + M.kin, reinterpret_cast<const InT *>(a.k) + (size_t)u * D, in_b, bar);
+                bulk_g2s(dst + M.vin, reinterpret_cast<const InT *>(a.v) + (size_t)u * D, in_b, bar);
+                if (KDA) {
+                    bulk_g2s(dst + M.gin, a.g + (size_t)u * D, 4 * D, bar);
+                    bulk_g2s(dst + M.gsum, w.gate_sum + (size_t)u * D, 8 * D, bar);
+                }
+                if (ncomp > 0) {
+                    bulk_g2s(dst + M.cidx, w.comp_index + (size_t)u * cis, 4 * cis, bar);
+                    if (ncr > 0) bulk_g2s(dst + M.crow, w.comp_row_vec + (size_t)u * ncr * D, 4 * D * ncr, bar);
+                    if (ncc > 0) bulk_g2s(dst + M.ccol, w.comp_col_vec + (size_t)u * ncc * D, 4 * D * ncc, bar);
+                }
                 advance();
+                if (u != early_u) {
+                    dst = acquire(u, -2);
+                    if (dst == nullptr) { fail(); return; }
+                    bar = &full[slot];
+                    mbar_arrive_expect_tx(bar, D * D);
+                    tma_load_2d(dst, &codes_map, 0, u * D, bar);
+                }
+                advance();
+                publish();
+                const int nchunks = (n_buf + E - 1) / E;
+                for (int c = 0; c < nchunks; ++c) {
+                    dst = acquire(u, -3 - c);
+                    if (dst == nullptr) { fail(); return; }
+                    const int e0 = c * E, ne = min(E, n_buf - e0);
+                    const size_t first = (size_t)u * w.window + e0;
+                    const uint32_t bd = 4u * ne * D, bk = (uint32_t)sizeof(KeyT) * ne * D;
+                    const uint32_t bg = KDA ? 0u : 4u * (uint32_t)align_up(ne, 4);
+                    bar = &full[slot];
+                    mbar_arrive_expect_tx(bar, bd + bk + bg);
+                    bulk_g2s(dst, w.buf_delta + first * D, bd, bar);
+                    bulk_g2s(dst + Sh::C_KEY, reinterpret_cast<const KeyT *>(w.buf_key) + first * D, bk, bar);
+                    if (!KDA) bulk_g2s(dst + Sh::C_GATE, w.buf_gate + (size_t)u * w.window_pad + e0, bg, bar);
+                    advance();
+                }
             }
+            // the next unit and its scalars (loads in flight until its record)
+            int un = -1;
+            if (k + 1 < rounds) {
+                un = u + grid;
+            } else if (draw) {
+                const unsigned long long r = tk % n_tk;
+                if (r < (unsigned long long)n_dyn) {
+                    un = rounds * grid + (int)r;
+                    tk = atomicAdd(tickets, 1ull);
+                } else {
+                    draw = false;
+                }
+            }
+            u = un;
+            if (u >= 0) fetch(u, cur);
         }
+        // no unit left: a record that says so
+        if (acquire(-1, -5) == nullptr) { fail(); return; }
+        stop(slot);
         return;
     }
 
@@ -256,45 +362,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     bool tc_inflight = false;                         // a pass was issued and not yet seen complete
     grid_dependency_wait();                           // the inputs and the buffer may still be in writing
     if (tid == 0) grid_dependents_launch();
-    int u = blockIdx.x;
-    float beta_n = 0.0f, g_n = 0.0f, gam_n = 0.0f;
-    double G_n = 0.0;
-    int fill_n = 0;
-    bool active_n = false;
-    if (u < units) {
-        fill_n = unit_fill(u);
-        active_n = unit_active(u);
-        beta_n = a.beta[u];
-        if (!KDA) {
-            g_n = a.g[u];
-            G_n = w.gate_sum[u] + (double)g_n;
-            gam_n = exp_of_double(G_n);
-        }
-    }
-    for (; u < units; u += gridDim.x) {
-        const float beta = beta_n;
-        const double Gs = G_n;                     // scalar gate: G_t
-        const float gam_s = gam_n;                 // scalar gate: gamma_t
-        const int n_buf = fill_n;
-        const bool active = active_n;
-        const int un = u + gridDim.x;
-        if (un < units) {                          // next unit's scalars, in flight meanwhile
-            fill_n = unit_fill(un);
-            active_n = unit_active(un);
-            beta_n = a.beta[un];
-            if (!KDA) { g_n = a.g[un]; G_n = w.gate_sum[un]; }
-        }
-        if (RAGGED && (!active || n_buf >= w.window || (kBoundsChecked && n_buf < 0))) {   // not decoded (nor loaded)
-            if (!KDA && un < units) {
-                G_n = G_n + (double)g_n;
-                gam_n = exp_of_double(G_n);
-            }
-            continue;
-        }
-        const int nchunks = (n_buf + E - 1) / E;
-
+    for (;;) {
         // ------------------------------------------------ A1: operand prep
         bool bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
+        const UnitRec r = rec[slot];
+        if (consumer_sync_or(bad || r.u < 0)) {   // a timeout, or no unit left
+            if (bad) report_error(w.err, LQ_DEVERR_TIMEOUT, -1, -6);
+            goto consumers_done;
+        }
+        const int u = r.u;
+        const float beta = r.beta;
+        const double Gs = r.G;                     // scalar gate: G_t
+        const float gam_s = r.gam;                 // scalar gate: gamma_t
+        const int n_buf = r.n_buf;
+        const int nchunks = (n_buf + E - 1) / E;
         const unsigned char *mp = ring + slot * kSlotBytes;
         const int meta_slot = slot;
         advance();
@@ -619,10 +700,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             w.gate_sum[u] = Gs;
         }
         if (RAGGED && tid == 64) a.fill[u] = n_buf + 1;
-        if (!KDA && un < units) {                  // next unit's G_t and gamma_t, off its critical path
-            G_n = G_n + (double)g_n;
-            gam_n = exp_of_double(G_n);
-        }
     }
 consumers_done:
     // every consumer warp gets here (normal end, or a timeout all of them saw at
