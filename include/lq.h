@@ -144,7 +144,8 @@ typedef struct lq_config {
 typedef struct lq_layout {
     size_t total_bytes;
     size_t err;           /* int32[64]: [0] LQ_DEVERR_*, [1] unit, [2] detail;
-                             [32..33] the windowed decode's unit-ticket counter */
+                             [32..33], [34..35] unit-ticket counters of the
+                             windowed decode and the window flush            */
     size_t codes;         /* int8  [N][d_v][d_k]                 window, naive    */
     size_t row_scale;     /* f32   [N][d_v]       sigma          window, naive    */
     size_t col_smooth;    /* f32   [N][d_k]       s              window           */

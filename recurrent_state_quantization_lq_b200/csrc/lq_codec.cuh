@@ -66,16 +66,27 @@ __device__ __forceinline__ void codec_store(Tile<D> &T, int u, const Views &w, i
 
     // ------------------------------------------------- 2a. compensator rows
     if (n_rows > 0) {
+        if (l2) {                                 // one branch per ranking, taken by every thread alike
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
-            float p = 0.0f;
+            for (int r = 0; r < NR; ++r) {
+                float p = 0.0f;
 #pragma unroll
-            for (int c = 0; c < NR; ++c) {
-                const float x = fabsf(T.at(r, c));
-                p = l2 ? p + x * x : fmaxf(p, x);
+                for (int c = 0; c < NR; ++c) {
+                    const float x = fabsf(T.at(r, c));
+                    p = p + x * x;
+                }
+                p = group_sum<16>(p);
+                if (tx == 0) sh_score[T.row(r)] = p;
             }
-            p = l2 ? group_sum<16>(p) : group_max<16>(p);
-            if (tx == 0) sh_score[T.row(r)] = p;
+        } else {
+#pragma unroll
+            for (int r = 0; r < NR; ++r) {
+                float p = 0.0f;
+#pragma unroll
+                for (int c = 0; c < NR; ++c) p = fmaxf(p, fabsf(T.at(r, c)));
+                p = group_max<16>(p);
+                if (tx == 0) sh_score[T.row(r)] = p;
+            }
         }
         tile_sync();
         const uint2 sel = select_top<D>(sh_score, n_rows);
@@ -84,14 +95,16 @@ __device__ __forceinline__ void codec_store(Tile<D> &T, int u, const Views &w, i
             for (int c = 0; c < 8; ++c)
                 if (c < n_rows) cidx[c] = sel_at(sel, c);
         }
+        // row i is held by the threads with ty = (i / 4) mod 16, as their row
+        // (i / 64) * 4 + i mod 4; only they store and clear it
+        for (int c = 0; c < n_rows; ++c) {
+            const int i = sel_at(sel, c);
+            if (((i >> 2) & 15) != ty) continue;
+            const int ri = ((i >> 6) << 2) | (i & 3);
+            float *dst = w.comp_row_vec + ((size_t)u * n_rows + c) * D;
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
-            int slot = -1;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                if (c < n_rows && sel_at(sel, c) == T.row(r)) slot = c;
-            if (slot >= 0) {
-                float *dst = w.comp_row_vec + ((size_t)u * n_rows + slot) * D;
+            for (int r = 0; r < NR; ++r) {
+                if (r != ri) continue;
 #pragma unroll
                 for (int g = 0; g < G; ++g)
                     *reinterpret_cast<float4 *>(dst + g * 64 + tx * 4) =
@@ -149,22 +162,22 @@ __device__ __forceinline__ void codec_store(Tile<D> &T, int u, const Views &w, i
         sh_rs[j] = __fdiv_rn(1.0f, s);          // applied as a multiplication
         if (w.col_smooth != nullptr) w.col_smooth[(size_t)u * D + j] = s;
     }
-    if (n_cols > 0) {
+    // column j is held by the threads with tx = (j / 4) mod 16, as their
+    // column (j / 64) * 4 + j mod 4; only they store and clear it
+    for (int cc = 0; cc < n_cols; ++cc) {
+        const int j = sel_at(csel, cc);
+        if (((j >> 2) & 15) != tx) continue;
+        const int cj = ((j >> 6) << 2) | (j & 3);
+        float *dst = w.comp_col_vec + ((size_t)u * n_cols + cc) * D;
 #pragma unroll
         for (int c = 0; c < NR; ++c) {
-            int slot = -1;
+            if (c != cj) continue;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc)
-                if (cc < n_cols && sel_at(csel, cc) == T.col(c)) slot = cc;
-            if (slot >= 0) {
-                float *dst = w.comp_col_vec + ((size_t)u * n_cols + slot) * D;
+            for (int g = 0; g < G; ++g)
+                *reinterpret_cast<float4 *>(dst + g * 64 + ty * 4) =
+                    make_float4(T.at(g * 4, c), T.at(g * 4 + 1, c), T.at(g * 4 + 2, c), T.at(g * 4 + 3, c));
 #pragma unroll
-                for (int g = 0; g < G; ++g)
-                    *reinterpret_cast<float4 *>(dst + g * 64 + ty * 4) =
-                        make_float4(T.at(g * 4, c), T.at(g * 4 + 1, c), T.at(g * 4 + 2, c), T.at(g * 4 + 3, c));
-#pragma unroll
-                for (int r = 0; r < NR; ++r) T.at(r, c) = 0.0f;
-            }
+            for (int r = 0; r < NR; ++r) T.at(r, c) = 0.0f;
         }
     }
     tile_sync();

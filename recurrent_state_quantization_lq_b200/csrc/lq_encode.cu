@@ -87,7 +87,7 @@ struct FlushShape {
     static constexpr int C_KEY = 4 * D * E;                         // chunk: deltas, keys, omega_j
     static constexpr int C_GATE = C_KEY + KB * D * E;
     // shared memory: barriers, ring, staged keys (two buffers), codec scratch
-    static constexpr int OFF_RING = 128;
+    static constexpr int OFF_RING = 128;        // barriers (64 bytes), unit records (64 bytes)
     static constexpr int OFF_STAGE = OFF_RING + kSlots * kSlotBytes;
     static constexpr int OFF_GAMMA = OFF_STAGE + (KDA ? 0 : 2 * kMaxChunk * D * 4);
     static constexpr int OFF_CODEC = OFF_GAMMA + 4 * D;
@@ -98,6 +98,17 @@ struct FlushShape {
 struct FlushMeta {
     int sig, s, gsum, cidx, crow, ccol, bytes;
 };
+
+// What the producer tells the tile threads about the unit whose meta segment
+// fills a slot (u < 0: no unit is left).
+struct FlushRec {
+    double gw;     // scalar gate: G at the window end
+    int u;
+    int pad;
+};
+
+// The flush's unit-ticket counter: a 64-bit word in the error region (int32 index).
+constexpr int kFlushTicketWord = 34;
 
 template <int D, bool KDA>
 __host__ __device__ FlushMeta flush_meta_layout(int ncr, int ncc, int cis) {
@@ -128,6 +139,7 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
     extern __shared__ __align__(128) unsigned char sm[];
     uint64_t *full = reinterpret_cast<uint64_t *>(sm);
     uint64_t *empty = full + kSlots;
+    FlushRec *rec = reinterpret_cast<FlushRec *>(empty + kSlots);   // one per ring slot
     unsigned char *ring = sm + Sh::OFF_RING;
     float *stage = reinterpret_cast<float *>(sm + Sh::OFF_STAGE);
     float *sgam = reinterpret_cast<float *>(sm + Sh::OFF_GAMMA);     // gamma_W per key channel
@@ -146,23 +158,52 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
     if (warp == kTile / 32) {
         if (lane != 0) return;
         const uint64_t stream_once = l2_policy_evict_first();
+        // Units: a CTA's first is its own index, the others come from a ticket
+        // counter in the workspace, so that a CTA that runs faster than the
+        // other one on its SM takes more of them.  A launch draws `units`
+        // tickets (one per unit past the CTAs' first ones, and one per CTA that
+        // finds none left), and launches of a state never draw at the same
+        // time, so one launch's tickets are consecutive counter values and
+        // t mod units takes each value once, whatever the counter held.
+        const int grid = (int)gridDim.x, n_dyn = units - grid;
+        unsigned long long *tickets = reinterpret_cast<unsigned long long *>(w.err + kFlushTicketWord);
         int slot = 0;
         uint32_t ph = 0;
+        uint32_t armed = 0;                        // slots filled at least once
         auto acquire = [&](int u, int detail) -> unsigned char * {
             if (!mbar_wait(&empty[slot], ph ^ 1u, kWaitBudgetCycles)) {
                 report_error(w.err, LQ_DEVERR_TIMEOUT, u, detail);
                 return nullptr;
             }
+            armed |= 1u << slot;
             return ring + slot * kSlotBytes;
         };
         auto advance = [&]() {
             if (++slot == kSlots) { slot = 0; ph ^= 1u; }
         };
-        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        // After a timed-out acquire: a meta slot still owed its record gets the
+        // end one, then wait (bounded) until every copy this thread started has
+        // landed, so that none writes into the shared memory of an exited CTA.
+        // Slot i was last filled in the round of parity ph (i < slot) or ph ^ 1.
+        auto fail = [&](int pend) {
+            if (pend >= 0) {
+                rec[pend].u = -1;
+                mbar_arrive(&full[pend]);
+            }
+            for (int i = 0; i < kSlots; ++i)
+                if (armed & (1u << i)) mbar_wait(&full[i], i < slot ? ph : (ph ^ 1u), kWaitBudgetCycles);
+        };
+        int u = (int)blockIdx.x;
+        unsigned long long tk = 0;
+        bool draw = n_dyn > 0;
+        if (draw) tk = atomicAdd(tickets, 1ull);   // the second unit's ticket
+        while (u >= 0) {
+            const double gw = KDA ? 0.0 : w.gate_sum[u];   // scalar gate: G at the window end
             unsigned char *dst = acquire(u, -1);
-            if (dst == nullptr) return;
+            if (dst == nullptr) { fail(-1); return; }
+            const int meta_slot = slot;
             uint64_t *bar = &full[slot];
-            mbar_arrive_expect_tx(bar, (uint32_t)M.bytes);
+            mbar_expect_tx(bar, (uint32_t)M.bytes);       // the arrival comes with the record
             bulk_g2s(dst + M.sig, w.row_scale + (size_t)u * D, 4 * D, bar);
             bulk_g2s(dst + M.s, w.col_smooth + (size_t)u * D, 4 * D, bar);
             if (KDA) bulk_g2s(dst + M.gsum, w.gate_sum + (size_t)u * D, 8 * D, bar);
@@ -173,14 +214,17 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
             }
             advance();
             dst = acquire(u, -2);
-            if (dst == nullptr) return;
+            if (dst == nullptr) { fail(meta_slot); return; }
             bar = &full[slot];
             mbar_arrive_expect_tx(bar, D * D);
             bulk_g2s_stream(dst, w.codes + (size_t)u * D * D, D * D, bar, stream_once);
             advance();
+            rec[meta_slot].gw = gw;
+            rec[meta_slot].u = u;
+            mbar_arrive(&full[meta_slot]);        // releases the record; the phase ends when the bytes land
             for (int c = 0; c < nchunks; ++c) {
                 dst = acquire(u, -3 - c);
-                if (dst == nullptr) return;
+                if (dst == nullptr) { fail(-1); return; }
                 const int e0 = c * E, ne = min(E, n_buf - e0);
                 const size_t first = (size_t)u * w.window + e0;
                 const uint32_t bd = 4u * ne * D, bk = (uint32_t)sizeof(KeyT) * ne * D;
@@ -193,7 +237,22 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
                 if (!KDA) bulk_g2s(dst + Sh::C_GATE, w.buf_gate + (size_t)u * w.window_pad + e0, bg, bar);
                 advance();
             }
+            // the next unit: its ticket was drawn a unit ago
+            u = -1;
+            if (draw) {
+                const int r = (int)(tk % (unsigned long long)units);
+                if (r < n_dyn) {
+                    u = grid + r;
+                    tk = atomicAdd(tickets, 1ull);
+                } else {
+                    draw = false;
+                }
+            }
         }
+        // no unit left: a record that says so
+        if (acquire(-1, -5) == nullptr) { fail(-1); return; }
+        rec[slot].u = -1;
+        mbar_arrive(&full[slot]);
         return;
     }
 
@@ -207,18 +266,19 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
     auto advance = [&]() {
         if (++slot == kSlots) { slot = 0; ph ^= 1u; }
     };
-    int u = blockIdx.x;
-    double G_n = (!KDA && u < units) ? w.gate_sum[u] : 0.0;
-    for (; u < units; u += gridDim.x) {
-        const double GW = G_n;                       // scalar gate: G at the window end
-        if (!KDA && u + (int)gridDim.x < units) G_n = w.gate_sum[u + gridDim.x];
-
-        // -------- dequantized window-start state plus compensators (undecayed)
+    for (;;) {
         bool bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
+        const int u = rec[slot].u;
+        const double GW = rec[slot].gw;              // scalar gate: G at the window end
+        if (tile_sync_or(bad || u < 0)) {           // a timeout, or no unit left
+            if (bad) report_error(w.err, LQ_DEVERR_TIMEOUT, -1, 0);
+            return;
+        }
+        // -------- dequantized window-start state plus compensators (undecayed)
         const unsigned char *mp = ring + slot * kSlotBytes;
         const int meta_slot = slot;
         advance();
-        bad |= !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
+        bad = !mbar_wait(&full[slot], ph, kWaitBudgetCycles);
         const int8_t *sQ = reinterpret_cast<const int8_t *>(ring + slot * kSlotBytes);
         const int q_slot = slot;
         advance();
@@ -244,27 +304,46 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
                     T.acc[r][g * 2 + 1] = make_float2((si * f2) * sc[g * 4 + 2], (si * f3) * sc[g * 4 + 3]);
                 }
             }
+            // The compensators as rank-1 terms on the packed FMAs, rows first,
+            // then columns: e_i k_c^T and v_c e_j^T.  fma(1, x, acc) = acc + x
+            // and fma(0, x, acc) = acc, so each element gets exactly the adds
+            // of its own compensators, in that order.
             if (ncomp > 0) {
                 const int32_t *cidx = reinterpret_cast<const int32_t *>(mp + M.cidx);
                 const float *crow = reinterpret_cast<const float *>(mp + M.crow);
                 const float *ccol = reinterpret_cast<const float *>(mp + M.ccol);
                 for (int c = 0; c < ncr; ++c) {
                     const int i = cidx[c];
+                    float2 kc[NR / 2];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float4 y = *reinterpret_cast<const float4 *>(crow + c * D + g * 64 + T.tx * 4);
+                        kc[g * 2 + 0] = make_float2(y.x, y.y);
+                        kc[g * 2 + 1] = make_float2(y.z, y.w);
+                    }
 #pragma unroll
                     for (int r = 0; r < NR; ++r) {
-                        if (T.row(r) == i) {
+                        const float e = T.row(r) == i ? 1.0f : 0.0f;
 #pragma unroll
-                            for (int cc = 0; cc < NR; ++cc) T.at(r, cc) += crow[c * D + T.col(cc)];
-                        }
+                        for (int m = 0; m < NR / 2; ++m) T.acc[r][m] = __ffma2_rn(make_float2(e, e), kc[m], T.acc[r][m]);
                     }
                 }
                 for (int c = 0; c < ncc; ++c) {
                     const int j = cidx[ncr + c];
+                    float2 ec[NR / 2];
 #pragma unroll
-                    for (int cc = 0; cc < NR; ++cc) {
-                        if (T.col(cc) == j) {
+                    for (int m = 0; m < NR / 2; ++m)
+                        ec[m] = make_float2(T.col(2 * m) == j ? 1.0f : 0.0f, T.col(2 * m + 1) == j ? 1.0f : 0.0f);
 #pragma unroll
-                            for (int r = 0; r < NR; ++r) T.at(r, cc) += ccol[c * D + T.row(r)];
+                    for (int g = 0; g < G; ++g) {
+                        const float4 x = *reinterpret_cast<const float4 *>(ccol + c * D + g * 64 + T.ty * 4);
+                        const float xr[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                        for (int rr = 0; rr < 4; ++rr) {
+#pragma unroll
+                            for (int m = 0; m < NR / 2; ++m)
+                                T.acc[g * 4 + rr][m] =
+                                    __ffma2_rn(make_float2(xr[rr], xr[rr]), ec[m], T.acc[g * 4 + rr][m]);
                         }
                     }
                 }
