@@ -112,9 +112,12 @@ enum { LQ_SELECT_L2 = 0, LQ_SELECT_MAXABS = 1 };
 enum { LQ_DTYPE_F32 = 0, LQ_DTYPE_BF16 = 1 };
 
 /* Device error codes in the workspace error word (lq_layout.err, int32[0]).
- * LQ_DEVERR_BOUNDS is raised only by the bounds-checked build of the library
- * (liblq_checked.so): a computed index outside its region, whose access was
- * skipped; lq_device_status() reports it as LQ_ERR_DEVICE. */
+ * LQ_DEVERR_BOUNDS: a computed index outside its region, whose access was
+ * skipped.  The bounds-checked build of the library (liblq_checked.so) checks
+ * the indices it derives from workspace contents; every build checks the unit
+ * tickets, which are out of range when a launch that ended on a device error
+ * left a ticket counter set (prefill clears it).  lq_device_status() reports
+ * it as LQ_ERR_DEVICE. */
 enum { LQ_DEVERR_NONE = 0, LQ_DEVERR_RANGE = 1, LQ_DEVERR_TIMEOUT = 2, LQ_DEVERR_WINDOW_FULL = 3,
        LQ_DEVERR_BOUNDS = 4 };
 
@@ -145,7 +148,8 @@ typedef struct lq_layout {
     size_t total_bytes;
     size_t err;           /* int32[64]: [0] LQ_DEVERR_*, [1] unit, [2] detail;
                              [32..33], [34..35] unit-ticket counters of the
-                             windowed decode and the window flush            */
+                             windowed decode and the window flush: zero
+                             between launches (prefill clears them)          */
     size_t codes;         /* int8  [N][d_v][d_k]                 window, naive    */
     size_t row_scale;     /* f32   [N][d_v]       sigma          window, naive    */
     size_t col_smooth;    /* f32   [N][d_k]       s              window           */

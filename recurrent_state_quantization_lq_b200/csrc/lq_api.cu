@@ -585,6 +585,11 @@ lq_status lq_device_status(lq_handle h, void *stream) {
         snprintf(buf, sizeof buf, "gate sum outside +-80 at unit %d, key channel %d: flush more often", word[1], word[2]);
         return fail(LQ_ERR_RANGE, buf);
     }
+    if (word[0] == LQ_DEVERR_BOUNDS && word[2] == -50) {
+        snprintf(buf, sizeof buf, "unit ticket out of range: a ticket counter was left set (after a device error); "
+                 "prefill the state again");
+        return fail(LQ_ERR_DEVICE, buf);
+    }
     if (word[0] == LQ_DEVERR_BOUNDS) {
         snprintf(buf, sizeof buf, "index out of range at unit %d (check site %d; bounds-checked build): the "
                  "workspace holds an inconsistent state", word[1], word[2]);

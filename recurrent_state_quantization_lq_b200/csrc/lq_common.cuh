@@ -112,6 +112,27 @@ __device__ __forceinline__ bool in_bounds(int32_t *err, long long idx, long long
     return false;
 }
 
+// --------------------------------------------------------------- unit tickets
+//
+// A launch that hands out n_dyn of its units by ticket draws from a 64-bit
+// counter in the workspace that is zero when it starts: ticket t < n_dyn names
+// the launch's dynamic unit t, any other names none.  Each of the grid CTAs
+// draws until it gets one that names none, so a launch draws exactly
+// n_dyn + grid tickets, and the CTA that draws the last one sets the counter
+// back to zero: no draw of this launch follows it, and the next launch draws
+// only after this one has completed.  A ticket past the last one means the
+// counter was not zero at the start (left by a launch that ended on a device
+// error); it is reported as LQ_DEVERR_BOUNDS.  Returns the unit number or -1.
+__device__ __forceinline__ int ticket_unit(unsigned long long t, int n_dyn, int grid, unsigned long long *counter,
+                                           int32_t *err) {
+    const unsigned long long last = (unsigned long long)n_dyn + (unsigned long long)grid - 1ull;
+    // a plain store: every draw of this launch came before this thread's last
+    // one, and an atomic exchange would hold the thread for its reply
+    if (t == last) *reinterpret_cast<volatile unsigned long long *>(counter) = 0ull;
+    else if (t > last) report_error(err, LQ_DEVERR_BOUNDS, -1, -50);
+    return t < (unsigned long long)n_dyn ? (int)t : -1;
+}
+
 // ------------------------------------------------- mbarrier + bulk async copies
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

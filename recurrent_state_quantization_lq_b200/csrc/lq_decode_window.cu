@@ -168,17 +168,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if (lane != 0) return;
         const uint32_t in_b = (uint32_t)sizeof(InT) * D;
         // Units: CTA b walks b, b + grid, ... through the whole rounds; the
-        // units of the last, partial round are handed out by a ticket counter
-        // in the workspace to the CTAs that get there first.  A launch then
-        // draws n_dyn + grid tickets (one per such unit, and one per CTA that
-        // finds none left), and launches of a state never draw at the same time
-        // (each draws only after the kernel before it has completed), so one
-        // launch's tickets are consecutive counter values: t mod (n_dyn + grid)
-        // runs over each value once, whatever the counter started from.
+        // units of the last, partial round are handed out by ticket (see
+        // ticket_unit) to the CTAs that get there first.  Each CTA draws at the
+        // start of its last whole-round unit, after the wait for the previous
+        // kernel, so no two launches draw at the same time.
         const int grid = (int)gridDim.x;
         const int rounds = units / grid;
         const int n_dyn = units - rounds * grid;
-        const unsigned long long n_tk = (unsigned long long)(n_dyn + grid);
         unsigned long long *tickets = reinterpret_cast<unsigned long long *>(w.err + kTicketWord);
         struct Scalars {
             int n;
@@ -324,9 +320,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if (k + 1 < rounds) {
                 un = u + grid;
             } else if (draw) {
-                const unsigned long long r = tk % n_tk;
-                if (r < (unsigned long long)n_dyn) {
-                    un = rounds * grid + (int)r;
+                const int r = ticket_unit(tk, n_dyn, grid, tickets, w.err);
+                if (r >= 0) {
+                    un = rounds * grid + r;
                     tk = atomicAdd(tickets, 1ull);
                 } else {
                     draw = false;

@@ -158,13 +158,10 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
     if (warp == kTile / 32) {
         if (lane != 0) return;
         const uint64_t stream_once = l2_policy_evict_first();
-        // Units: a CTA's first is its own index, the others come from a ticket
-        // counter in the workspace, so that a CTA that runs faster than the
-        // other one on its SM takes more of them.  A launch draws `units`
-        // tickets (one per unit past the CTAs' first ones, and one per CTA that
-        // finds none left), and launches of a state never draw at the same
-        // time, so one launch's tickets are consecutive counter values and
-        // t mod units takes each value once, whatever the counter held.
+        // Units: a CTA's first is its own index, the others are handed out by
+        // ticket (see ticket_unit), so that a CTA that runs faster than the
+        // other one on its SM takes more of them.  The kernel before a flush
+        // has completed when it starts, so no two launches draw at the same time.
         const int grid = (int)gridDim.x, n_dyn = units - grid;
         unsigned long long *tickets = reinterpret_cast<unsigned long long *>(w.err + kFlushTicketWord);
         int slot = 0;
@@ -240,8 +237,8 @@ __global__ void __launch_bounds__(kFlushThreads, 2) flush_kernel(EncodeArgs a) {
             // the next unit: its ticket was drawn a unit ago
             u = -1;
             if (draw) {
-                const int r = (int)(tk % (unsigned long long)units);
-                if (r < n_dyn) {
+                const int r = ticket_unit(tk, n_dyn, grid, tickets, w.err);
+                if (r >= 0) {
                     u = grid + r;
                     tk = atomicAdd(tickets, 1ull);
                 } else {

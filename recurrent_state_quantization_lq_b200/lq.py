@@ -28,7 +28,7 @@ SELECT = {"l2": 0, "maxabs": 1}
 DTYPE = {torch.float32: 0, torch.bfloat16: 1}
 ABSENT = ctypes.c_size_t(-1).value
 
-LQ_DEVERR_BOUNDS = 4   # device error code of the bounds-checked build
+LQ_DEVERR_BOUNDS = 4   # device error code: an index out of range (checked build; unit tickets in every build)
 
 STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED", 3: "LQ_ERR_WORKSPACE",
                 4: "LQ_ERR_WINDOW_FULL", 5: "LQ_ERR_RANGE", 6: "LQ_ERR_CUDA", 7: "LQ_ERR_DEVICE",

@@ -73,3 +73,47 @@ def test_inputs_written_by_the_previous_kernel(batch):
         torch.mul(x, 1, out=dst)
     assert torch.equal(a.decode_step(*bufs), b.decode_step(*src))
     assert a.device_status() == lq.LQ_OK and b.device_status() == lq.LQ_OK
+
+
+@pytest.mark.parametrize("batch,window", [(37, 8), (40, 8), (2, 8)])
+def test_ticket_counters_return_to_zero(batch, window):
+    """The decode and the flush hand out units by ticket counters kept in the
+    error region (int32 words 32-35).  Every launch starts from zero and the
+    CTA that draws its last ticket sets the counter back, so both read zero
+    after every decode and flush, whatever the grid; and a checkpoint taken
+    between launches resumes on any number of SMs.  On 148 SMs (592 decode
+    CTAs, 296 flush CTAs) 37 x 32 = 1184 units fill two whole decode rounds,
+    40 x 32 leaves a partial one of 96, and 2 x 32 needs no ticket at all."""
+    a, b = _pair(batch, 13, same=True)
+    tb = inputs.tokens_on_device(7, 2 * window, batch, H, D, D, False, torch.bfloat16, DEV)
+    zero = torch.zeros(4, dtype=torch.int32)
+    for t in range(2 * window):
+        oa = a.decode_step(*_tok(tb, t))
+        assert torch.equal(a.view("err")[32:36].cpu(), zero), t
+        assert torch.equal(oa, b.decode_step(*_tok(tb, t))), t
+        if t % window == window - 1:
+            a.flush()
+            b.flush()
+            assert torch.equal(a.view("err")[32:36].cpu(), zero), t
+    assert a.device_status() == lq.LQ_OK and b.device_status() == lq.LQ_OK
+
+
+def test_ticket_counter_left_set_is_reported():
+    """A counter that is not zero when a launch starts (as a launch that ended
+    on a device error may leave it) hands out tickets past the launch's range:
+    the kernels report LQ_DEVERR_BOUNDS instead of going on silently, and a
+    prefill clears the counters again."""
+    batch = 40                                          # decode and flush both draw
+    a, _ = _pair(batch, 14)
+    tb = inputs.tokens_on_device(8, 2, batch, H, D, D, False, torch.bfloat16, DEV)
+    big = torch.tensor([0, 1 << 20, 0, 1 << 20], dtype=torch.int32, device=DEV)
+    a.view("err")[32:36].copy_(big)
+    a.decode_step(*_tok(tb, 0))
+    assert a.device_status() == lq.LQ_ERR_DEVICE
+    err = a.view("err")[:3].cpu()
+    assert int(err[0]) == lq.LQ_DEVERR_BOUNDS and int(err[2]) == -50
+    a.prefill(None)
+    assert torch.equal(a.view("err")[32:36].cpu(), torch.zeros(4, dtype=torch.int32))
+    a.decode_step(*_tok(tb, 1))
+    a.flush()
+    assert a.device_status() == lq.LQ_OK
