@@ -725,7 +725,7 @@ def ragged_phases(dev, wl, L: int = 4, reps: int = 20) -> list[dict]:
         for st in stk.states:
             assert st.device_status(stream) == lq.LQ_OK, lq.last_error()
         if rag:
-            fills = torch.stack([st.fills() for st in stk.states]).view(L, B, wl.heads)
+            fills = torch.stack([st.fills() for st in stk.states]).view(L, B, wl.heads).to(offset.device)
             want = offset if stagger else torch.zeros_like(offset)
             assert bool((fills == want.view(1, B, 1)).all()), "phases drifted"
         ms = e0.elapsed_time(e1) / reps                   # W tokens of every sequence, every layer
@@ -765,7 +765,7 @@ def prefill_timing(dev, wl, T: int | None = None, reps: int = 5) -> list[dict]:
         f32.prefill(None)
         for t in range(T):
             f32.decode_step(tb.q[t], tb.k[t], tb.v[t], tb.g[t], tb.beta[t], out=out[t])
-        win.prefill(f32.read("state_f32", device=f32.device))
+        win.prefill(f32.view("state_f32"))               # the FP32 state in place (no copy, no sync)
 
     rows = []
     flop = (6 + (1 if wl.per_channel_gate else 0)) * d * d          # per token and head
