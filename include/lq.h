@@ -61,7 +61,9 @@
  *    on the calling thread is lq_last_error_string().  Errors found on the
  *    device (a gate sum out of the safe range, a bounded wait that expired)
  *    are recorded in the workspace's error word and reported by
- *    lq_device_status().  No kernel traps or asserts.
+ *    lq_device_status().  No kernel traps or asserts.  A state whose error
+ *    word is set is to be prefilled again before further use: the launch that
+ *    recorded the error may have left it partly updated.
  *  - Tracing.  Every call that enqueues device work opens an NVTX range named
  *    after the call, so timeline tools group its kernels under it.
  *  - Window phase.  By default all sequences of a handle share one window
